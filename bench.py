@@ -1,0 +1,581 @@
+#!/usr/bin/env python
+"""Bench: one routed MoE layer over 2-bit (Q2) block-quantized experts on B200.
+
+Headline workload: the full-size decode/verify layer (hidden 2048, 512 routed
+experts, top-10 + 1 shared, intermediate 512, T = 3 tokens, uniform router).
+A step is one pass of the whole layer (router GEMV, top-k, dispatch, gate/up +
+SwiGLU, down, combine) over one batch of 3 synthetic tokens.  The same run
+also measures the 1024-token prefill chunk with the Zipf-skewed router and
+reports it under "prefill_t1024".
+
+Timing: steps are captured in CUDA graphs and timed with CUDA events on the
+launch stream, with a barrier + synchronize on both sides (max over ranks for
+N > 1).  Decode steps rotate over 24 distinct copies of the layer weights
+(11.8 GB) and 64 input slots, so a step never finds its weights in the 126 MB
+L2; a prefill step reads all 513 experts (> L2).
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (the
+reference arm of this benchmark; there is no runnable upstream code).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at decode T=3 and prefill T=1024; % of HBM/tensor roofline"
+EXPERT_BYTES = 983040          # one Q2 expert at hidden 2048 / intermediate 512
+SPEC_HBM_GBS = 8000.0          # headline HBM figure
+SPEC_BF16_TFLOPS = 2250.0      # dense bf16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=24000)
+    ap.add_argument("--warmup", type=int, default=240)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--prefill-steps", type=int, default=40)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+
+class ClockSampler:
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+
+def make_layer_sets(cfg, n_distinct: int, n_sets: int, seed: int, device):
+    """n_sets device copies of n_distinct seeded layers (distinct memory -> no L2 reuse)."""
+    import torch
+
+    from bit_block_quantized_moe_b200 import Q2MoeLayer
+    from gen import make_layer
+
+    base = []
+    for l in range(n_distinct):
+        w = make_layer(cfg, seed=seed, layer=l)
+        base.append(Q2MoeLayer(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, w["router_w"], w["router_b"],
+                               w["experts"], w["shared"], device=device))
+    sets = []
+    for i in range(n_sets):
+        b = base[i % n_distinct]
+        if i < n_distinct:
+            sets.append((b.router_w, b.router_b, b.experts, b.shared))
+        else:
+            sets.append((b.router_w.clone(), None if b.router_b is None else b.router_b.clone(), b.experts.clone(),
+                         b.shared.clone()))
+    torch.cuda.synchronize()
+    return base[0].dims, sets
+
+
+def capture(fn, n_steps, stream):
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        for i in range(n_steps):
+            fn(i)
+    return g
+
+
+def time_graph_steps(fn, K, W, stream, world, chunk=240, sampler=None):
+    """Warm up W steps, then time exactly K steps (graphs of <= chunk steps); returns seconds (max over ranks)."""
+    import torch
+
+    gw = capture(fn, max(1, min(W, chunk)), stream) if W > 0 else None
+    full, rem = divmod(K, chunk)
+    g_full = capture(fn, chunk, stream) if full else None
+    g_rem = capture(fn, rem, stream) if rem else None
+    torch.cuda.synchronize()
+    if gw is not None:
+        done = 0
+        while done < W:
+            gw.replay()
+            done += max(1, min(W, chunk))
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        start.record(stream)
+        for _ in range(full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    secs = start.elapsed_time(end) / 1e3
+    del gw, g_full, g_rem
+    return max_over_ranks(secs, world)
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def traced_kernel_ms(fn, n_steps, kernel_id, stream):
+    """Average duration of one library kernel over n_steps graph-captured steps,
+    from CUDA events the library records around that kernel."""
+    import torch
+
+    import bit_block_quantized_moe_b200 as M
+
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(n_steps)]
+
+    def traced(i):
+        M.moe_trace_kernel(kernel_id, evs[i][0], evs[i][1])
+        fn(i)
+        M.moe_trace_kernel(-1)
+
+    g = capture(traced, n_steps, stream)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    del g
+    return sum(ms) / len(ms)
+
+
+def gpu_uuid(dev):
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import bit_block_quantized_moe_b200 as M
+    from gen import CONFIGS, make_x
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream()
+    K, W = args.steps, max(args.warmup, 3)
+
+    # ---- decode layer, T = 3 -------------------------------------------------------
+    cfg = CONFIGS[1]
+    T, H = cfg.tokens, cfg.hidden
+    n_sets, n_slots = 24, 64
+    dims, sets = make_layer_sets(cfg, 4, n_sets, args.seed, dev)
+    xs = torch.stack([torch.from_numpy(make_x(T, H, seed=1000 * (rank + 1) + s).view(np.int16)) for s in range(n_slots)])
+    xs = xs.to(dev)
+    outs = torch.empty_like(xs)
+    ws = torch.empty(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
+    idx_all = torch.empty((n_sets * n_slots, T, cfg.top_k), dtype=torch.int32, device=dev)
+    w_all = torch.empty((n_sets * n_slots, T, cfg.top_k), dtype=torch.float32, device=dev)
+
+    def step(i):
+        rw, rb, ex, sh = sets[i % n_sets]
+        s = i % n_slots
+        M.moe_layer_forward(dims, xs[s], rw, rb, ex, sh, outs[s], T, ws, stream=stream)
+
+    # routing of every (set, slot) pair for the algorithmic-byte count
+    with torch.cuda.stream(stream):
+        for si in range(n_sets):
+            for s in range(n_slots):
+                rw, rb, ex, sh = sets[si]
+                M.moe_route(dims, xs[s], rw, rb, T, idx_all[si * n_slots + s], w_all[si * n_slots + s], ws,
+                            stream=stream)
+    torch.cuda.synchronize()
+    idx_np = idx_all.cpu().numpy()
+    touched = np.array([len(np.unique(idx_np[p])) for p in range(n_sets * n_slots)])
+
+    def step_pair(i):
+        return (i % n_sets) * n_slots + (i % n_slots)
+
+    sampler = ClockSampler(gpu_uuid(dev)) if rank == 0 else None
+    secs = time_graph_steps(step, K, W, stream, world, sampler=sampler)
+    ms_per_step = secs * 1e3 / K
+    value = world * T * K / secs
+
+    avg_touched = float(np.mean([touched[step_pair(i)] for i in range(min(K, 24 * 64 * 4))]))
+    expert_bytes = (avg_touched + 1) * EXPERT_BYTES
+    layer_bytes = expert_bytes + cfg.n_experts * H * 4 + 2 * T * H * 2
+    # dominant kernel: the gate/up projection (2/3 of the expert bytes)
+    n_trace = min(240, max(24, K))
+    gu_ms = traced_kernel_ms(step, n_trace, M.MOE_KERNEL["gate_up"], stream)
+    gu_bytes = (avg_touched + 1) * EXPERT_BYTES * 2 / 3 + T * H * 2
+    hbm_peak = float(peaks["hbm_gbs"])
+    gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
+    layer_gbs = layer_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API, host buffers --------------------------------
+    n_e2e = min(K, 2000)
+    xh = torch.empty((n_slots, T, H), dtype=torch.int16).pin_memory()
+    xh.copy_(xs.cpu())
+    oh = torch.empty((n_slots, T, H), dtype=torch.int16).pin_memory()
+    xd = torch.empty((T, H), dtype=torch.int16, device=dev)
+    od = torch.empty((T, H), dtype=torch.int16, device=dev)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            xd.copy_(xh[i], non_blocking=True)
+            rw, rb, ex, sh = sets[i % n_sets]
+            M.moe_layer_forward(dims, xd, rw, rb, ex, sh, od, T, ws, stream=stream)
+            oh[i].copy_(od, non_blocking=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(n_e2e):
+            s = i % n_slots
+            xd.copy_(xh[s], non_blocking=True)
+            rw, rb, ex, sh = sets[i % n_sets]
+            M.moe_layer_forward(dims, xd, rw, rb, ex, sh, od, T, ws, stream=stream)
+            oh[s].copy_(od, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    e2e_value = world * T * n_e2e / e2e_secs
+    M.moe_check_status(ws)
+
+    result = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded: x~N(0,1) bf16, router N(0,0.02) fp32, Q2 codes uniform, scales |N(0,0.02)| fp16)",
+        "config": {
+            "workload": "decode layer: hidden 2048, 512 routed experts top-10 + 1 shared, intermediate 512, "
+                        "SwiGLU, Q2 32-weight blocks, T=3 tokens, uniform router",
+            "global_batch": T * world,
+            "seq_len": T,
+            "parallelism": f"{world} independent token-parallel replicas, no collective",
+            "l2": "24 rotating weight copies (11.8 GB) and 64 input slots: inputs larger than L2",
+            "touched_experts_per_step": avg_touched,
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "gate_up (expert gate/up projection + SwiGLU)",
+            "achieved": gu_gbs,
+            "peak": hbm_peak,
+            "unit": "GB/s",
+            "frac": gu_gbs / hbm_peak,
+            "traffic": None,
+            "peak_source": f"{peak_src} hbm_gbs",
+            "kernel_ms": gu_ms,
+            "algorithmic_bytes": gu_bytes,
+        },
+        "layer_roofline": {
+            "bytes_per_step": layer_bytes,
+            "achieved_gbs": layer_gbs,
+            "frac_of_measured": layer_gbs / hbm_peak,
+            "frac_of_8tbs": layer_gbs / SPEC_HBM_GBS,
+        },
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+                "d2h_bytes_per_step": T * H * 2, "steps": n_e2e},
+        "gpu_launches": 7 * K,
+    }
+    if sampler is not None:
+        result["clocks"] = sampler.summary()
+
+    # ---- prefill chunk, T = 1024 ---------------------------------------------------------
+    if not args.no_prefill:
+        result["prefill_t1024"] = run_prefill(args, world, rank, dev, stream, peaks, peak_src)
+    return result
+
+
+def run_prefill(args, world, rank, dev, stream, peaks, peak_src):
+    import numpy as np
+    import torch
+
+    import bit_block_quantized_moe_b200 as M
+    from gen import CONFIGS, make_x
+
+    cfg = CONFIGS[2]
+    T, H = cfg.tokens, cfg.hidden
+    dims, sets = make_layer_sets(cfg, 1, 1, args.seed, dev)
+    rw, rb, ex, sh = sets[0]
+    n_slots = 4
+    xs = torch.stack([torch.from_numpy(make_x(T, H, seed=2000 * (rank + 1) + s).view(np.int16))
+                      for s in range(n_slots)]).to(dev)
+    outs = torch.empty_like(xs)
+    ws = torch.empty(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
+    idx = torch.empty((n_slots, T, cfg.top_k), dtype=torch.int32, device=dev)
+    wts = torch.empty((n_slots, T, cfg.top_k), dtype=torch.float32, device=dev)
+
+    def step(i):
+        s = i % n_slots
+        M.moe_layer_forward(dims, xs[s], rw, rb, ex, sh, outs[s], T, ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for s in range(n_slots):
+            M.moe_route(dims, xs[s], rw, rb, T, idx[s], wts[s], ws, stream=stream)
+    torch.cuda.synchronize()
+    touched = float(np.mean([len(np.unique(idx[s].cpu().numpy())) for s in range(n_slots)]))
+    K = args.prefill_steps
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=20)
+    ms = secs * 1e3 / K
+    bytes_ = (touched + 1) * EXPERT_BYTES + cfg.n_experts * H * 4 + 2 * T * H * 2
+    flops = T * (cfg.top_k + 1) * 6 * H * cfg.inter + 2 * T * H * cfg.n_experts
+    hbm = float(peaks["hbm_gbs"])
+    tflops = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    t_roof = max(bytes_ / (hbm * 1e9), flops / (tflops * 1e12))
+    t_roof_spec = max(bytes_ / (SPEC_HBM_GBS * 1e9), flops / (SPEC_BF16_TFLOPS * 1e12))
+    gu_ms = traced_kernel_ms(step, min(K, 8), M.MOE_KERNEL["gate_up"], stream)
+    gu_flops = (T * cfg.top_k + T) * 4 * H * cfg.inter
+    return {
+        "value": world * T * K / secs,
+        "unit": "tokens/s",
+        "ms_per_step": ms,
+        "steps": K,
+        "workload": "prefill chunk: T=1024, Zipf(s=1.1) router bias (hottest expert ~100 slots), same layer dims",
+        "touched_experts": touched,
+        "bytes_per_step": bytes_,
+        "flops_per_step": flops,
+        "binding": "hbm" if bytes_ / (hbm * 1e9) >= flops / (tflops * 1e12) else "tensor",
+        "roofline_frac_of_measured": t_roof / (ms * 1e-3),
+        "roofline_frac_of_spec": t_roof_spec / (ms * 1e-3),
+        "gate_up_kernel_ms": gu_ms,
+        "gate_up_tflops": gu_flops / (gu_ms * 1e-3) / 1e12,
+        "peak_source": peak_src,
+    }
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+
+
+def oracle_decode_tokens_per_s(budget_s: float, seed: int, max_tokens=4096):
+    """Time the fp64 oracle on decode-layer tokens (config-1 layer) for about budget_s seconds."""
+    import numpy as np
+
+    import oracle
+    from gen import CONFIGS, make_layer, make_x
+
+    cfg = CONFIGS[1]
+    w = make_layer(cfg, seed=seed, layer=0)
+    nthr = oracle.num_threads()
+    batch = max(3, nthr)
+    done, t_used, i = 0, 0.0, 0
+    while t_used < budget_s and done < max_tokens:
+        x = make_x(batch, cfg.hidden, seed=5000 + i)
+        t0 = time.perf_counter()
+        oracle.layer(x, w["router_w"], w["router_b"], w["experts"], w["shared"], cfg.top_k, cfg.inter)
+        t_used += time.perf_counter() - t0
+        done += batch
+        i += 1
+    return done / t_used, nthr, done, t_used
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import numpy as np
+
+    import oracle
+    from gen import CONFIGS, make_layer, make_x
+
+    cfg = CONFIGS[1]
+    w = make_layer(cfg, seed=args.seed, layer=0)
+    T = cfg.tokens
+    nthr = oracle.num_threads()
+
+    def one(i):
+        x = make_x(T, cfg.hidden, seed=7000 + i)
+        oracle.layer(x, w["router_w"], w["router_b"], w["experts"], w["shared"], cfg.top_k, cfg.inter)
+
+    budget = 150.0
+    t0 = time.perf_counter()
+    for i in range(max(args.warmup, 3)):
+        one(i)
+        if time.perf_counter() - t0 > 30:
+            break
+    steps, t_used = 0, 0.0
+    while steps < args.steps and t_used < budget:
+        a = time.perf_counter()
+        one(steps)
+        t_used += time.perf_counter() - a
+        steps += 1
+    value = steps * T / t_used
+    sample = (f"{steps} decode steps of T=3 tokens each (the full decode workload per step), "
+              f"capped at {budget:.0f} s of oracle time")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_used * 1e3 / steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "decode layer: hidden 2048, 512 routed experts top-10 + 1 shared, intermediate 512, "
+                               "SwiGLU, Q2 32-weight blocks, T=3 tokens, uniform router",
+                   "impl": "fp64 CPU oracle (plain C, OpenMP over tokens)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(nthr, T), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, world, rank)
+        if rank == 0:
+            print(json.dumps(res))
+        return
+    import torch
+
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    import __graft_entry__
+
+    __graft_entry__.build()
+    res = run_ours(args, world, rank, local)
+    if rank == 0 and not args.no_cpu:
+        tps, nthr, ntok, tsec = oracle_decode_tokens_per_s(12.0, args.seed)
+        res["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthr, "kind": "oracle",
+                               "sample": f"{ntok} decode-layer tokens (config-1 layer) in {tsec:.1f} s, "
+                                         f"OpenMP over tokens"}
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

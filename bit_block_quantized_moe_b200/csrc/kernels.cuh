@@ -1,0 +1,49 @@
+// Internal launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Workspace regions for one moe_layer_forward / moe_route call (device pointers).
+struct Workspace {
+  uint32_t *status;        // sticky status word
+  uint32_t *zero_begin;    // [zero_begin, zero_begin + zero_words) is cleared by the router kernel
+  size_t zero_words;
+  uint32_t *done_counter;  // last-block counter of the dispatch scan (inside the zeroed range)
+  uint32_t *n_items;
+  uint32_t *bitmap;        // [E][words] token-membership bits per expert (inside the zeroed range)
+  uint32_t *wprefix;       // [E][words] exclusive popcount prefix per word
+  int32_t *counts;         // [E]
+  int32_t *offsets;        // [E + 1]
+  float *logits;           // [T][E]
+  int32_t *idx;            // [T][k]
+  float *w;                // [T][k]
+  int32_t *slot_pos;       // [T*k]: sorted position of slot (t, j)
+  int32_t *sorted_tok;     // [T*k + T]: token of each sorted position (shared slots last)
+  float *sorted_w;         // [T*k + T]
+  int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)
+  uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position
+  float *y;                // [T*k + T][H] fp32 expert outputs by sorted position
+  int words;               // ceil(T / 32)
+  int max_items;
+};
+
+// Profiling hook (moe_trace_kernel): records the caller's events around kernel `id`.
+void trace_mark(int id, bool after, cudaStream_t s);
+
+size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws);
+
+cudaError_t launch_pack(const uint8_t *canon, uint8_t *packed, int n_experts, const PackedGeom &G,
+                        size_t canon_stride, cudaStream_t s);
+cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias, int T,
+                         const Workspace &ws, bool with_dispatch_bits, cudaStream_t s);
+cudaError_t launch_dispatch_bits(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s);
+cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s);
+cudaError_t launch_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
+                           const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
+cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s);
+cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,
+                                    cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,509 @@
+// Repacking, routing, dispatch, combine and the between-layer RMSNorm (sm_100a).
+//
+// Routing follows the problem statement of the pages: each token goes to
+// top_k of n_experts routed experts plus one shared expert (Strata tuning
+// page, section 2 model table; devlabs page, section 1).  The selection rule
+// (largest logit, ties to the lower index), the fp32 softmax over the
+// selected set and the bias placement are this library's stated readings.
+#include <float.h>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// moe_pack_q2: canonical 10-byte blocks -> fragment-ordered units.
+//
+// A unit is a 16-row tile.  Gate/up unit u: tile rows 0-7 are gate rows
+// 8u..8u+7, tile rows 8-15 are up rows 8u..8u+7.  Down unit u: tile rows are
+// down rows 16u..16u+15.  Along K the unit is cut into groups of 4 blocks
+// (128 weights); a group stores 32 lanes x 16 bytes of codes followed by
+// 8 x 16 bytes of scales.  Lane (g = lane/4, c = lane%4) owns tile rows g and
+// g+8; its word for block b holds, for k16 step s in {0,1}, the k pairs
+// (4c, 4c+1) and (4c+2, 4c+3) of both rows: pair p = 4s + P with
+// P = 0: row g, k 4c;  P = 1: row g+8, k 4c;  P = 2: row g, k 4c+2;  P = 3: row g+8, k 4c+2
+// (k relative to 32b + 16s); the even-k code sits at bit 2p, the odd-k code
+// at bit 16+2p.  Scales: for g in 0..7, block 0..3: (d[row g], d[row g+8]).
+__global__ void pack_q2_kernel(const uint8_t *__restrict__ canon, uint8_t *__restrict__ packed, int n_experts,
+                               PackedGeom G, size_t canon_stride) {
+  const int ug_per_expert = G.gu_units * G.gu_groups + G.dn_units * G.dn_groups;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long total = (long long)n_experts * ug_per_expert * 32;
+  if (tid >= total) return;
+  const int lane = (int)(tid & 31);
+  const long long r = tid >> 5;
+  const int ug = (int)(r % ug_per_expert);
+  const int e = (int)(r / ug_per_expert);
+  const uint8_t *ce = canon + (size_t)e * canon_stride;
+  uint8_t *pe = packed + (size_t)e * G.expert_bytes;
+  const size_t gu_mat_bytes = (size_t)G.I * G.H / kQBlock * kCanonBlockBytes;
+  const bool is_gu = ug < G.gu_units * G.gu_groups;
+  int unit, grp, ncols;
+  uint8_t *dst;
+  if (is_gu) {
+    unit = ug / G.gu_groups;
+    grp = ug % G.gu_groups;
+    ncols = G.H;
+    dst = pe + (size_t)unit * G.gu_unit_bytes + (size_t)grp * kGroupBytes;
+  } else {
+    const int v = ug - G.gu_units * G.gu_groups;
+    unit = v / G.dn_groups;
+    grp = v % G.dn_groups;
+    ncols = G.I;
+    dst = pe + G.gu_bytes + (size_t)unit * G.dn_unit_bytes + (size_t)grp * kGroupBytes;
+  }
+  const int nb = ncols / kQBlock;
+  auto row_ptr = [&](int rho) -> const uint8_t * {
+    if (is_gu) {
+      return rho < 8 ? ce + (size_t)(8 * unit + rho) * nb * kCanonBlockBytes
+                     : ce + gu_mat_bytes + (size_t)(8 * unit + rho - 8) * nb * kCanonBlockBytes;
+    }
+    return ce + 2 * gu_mat_bytes + (size_t)(16 * unit + rho) * nb * kCanonBlockBytes;
+  };
+  auto code = [&](int rho, int k) -> uint32_t {
+    const uint8_t *blk = row_ptr(rho) + (size_t)(k / kQBlock) * kCanonBlockBytes;
+    const int j = k % kQBlock;
+    return (blk[2 + (j >> 2)] >> (2 * (j & 3))) & 3u;
+  };
+  const int g = lane >> 2, c = lane & 3;
+  uint32_t words[4];
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    const int b = grp * 4 + wi;
+    uint32_t w = 0;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const int s = p >> 2, P = p & 3;
+      const int rho = g + 8 * (P & 1);
+      const int k = 32 * b + 16 * s + 4 * c + 2 * (P >> 1);
+      w |= code(rho, k) << (2 * p);
+      w |= code(rho, k + 1) << (16 + 2 * p);
+    }
+    words[wi] = w;
+  }
+  *reinterpret_cast<uint4 *>(dst + lane * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+  if (lane < 8) {
+    uint32_t sc[4];
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      const int b = grp * 4 + wi;
+      const uint8_t *b0 = row_ptr(lane) + (size_t)b * kCanonBlockBytes;
+      const uint8_t *b1 = row_ptr(lane + 8) + (size_t)b * kCanonBlockBytes;
+      const uint32_t d0 = b0[0] | ((uint32_t)b0[1] << 8);
+      const uint32_t d1 = b1[0] | ((uint32_t)b1[1] << 8);
+      sc[wi] = d0 | (d1 << 16);
+    }
+    *reinterpret_cast<uint4 *>(dst + kGroupCodeBytes + lane * 16) = make_uint4(sc[0], sc[1], sc[2], sc[3]);
+  }
+}
+
+cudaError_t launch_pack(const uint8_t *canon, uint8_t *packed, int n_experts, const PackedGeom &G,
+                        size_t canon_stride, cudaStream_t s) {
+  const long long ug = (long long)G.gu_units * G.gu_groups + (long long)G.dn_units * G.dn_groups;
+  const long long threads = (long long)n_experts * ug * 32;
+  const int bs = 256;
+  const long long blocks = (threads + bs - 1) / bs;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  pack_q2_kernel<<<(unsigned)blocks, bs, 0, s>>>(canon, packed, n_experts, G, canon_stride);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Router logits, fp32 accumulation.  Also clears the dispatch bit map for this
+// call (stream order puts the clear before the top-k kernel's atomics).
+
+__device__ __forceinline__ void clear_range(uint32_t *p, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
+}
+
+// Few tokens (T <= 8): one warp per expert row, 128-bit streaming loads of Wr.
+__global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t *__restrict__ x,
+                                                                   const float *__restrict__ Wr,
+                                                                   const float *__restrict__ bias, int T, int H,
+                                                                   int E, float *__restrict__ logits,
+                                                                   uint32_t *zero_p, size_t zero_n) {
+  clear_range(zero_p, zero_n);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (e >= E) return;
+  const float *wrow = Wr + (size_t)e * H;
+  float acc[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+#pragma unroll 4
+  for (int k = lane * 4; k < H; k += 128) {
+    const uint4 wv = ldg_nc_v4(wrow + k);
+    const float w0 = __uint_as_float(wv.x), w1 = __uint_as_float(wv.y), w2 = __uint_as_float(wv.z),
+                w3 = __uint_as_float(wv.w);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (t < T) {
+        const uint2 xv = *reinterpret_cast<const uint2 *>(x + (size_t)t * H + k);
+        float a = acc[t];
+        a = fmaf(__uint_as_float(xv.x << 16), w0, a);
+        a = fmaf(__uint_as_float(xv.x & 0xffff0000u), w1, a);
+        a = fmaf(__uint_as_float(xv.y << 16), w2, a);
+        a = fmaf(__uint_as_float(xv.y & 0xffff0000u), w3, a);
+        acc[t] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+  }
+  if (lane == 0) {
+    const float b = bias ? bias[e] : 0.f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (t < T) logits[(size_t)t * E + e] = acc[t] + b;
+  }
+}
+
+// Many tokens: 64 tokens x 64 experts per CTA, fp32 FMA tiles through shared memory.
+__global__ void __launch_bounds__(256) router_logits_tiled_kernel(const uint16_t *__restrict__ x,
+                                                                   const float *__restrict__ Wr,
+                                                                   const float *__restrict__ bias, int T, int H,
+                                                                   int E, float *__restrict__ logits,
+                                                                   uint32_t *zero_p, size_t zero_n) {
+  clear_range(zero_p, zero_n);
+  __shared__ float xs[32][68];
+  __shared__ float ws[32][68];
+  const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < H; k0 += 32) {
+    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
+      const int row = i >> 5, kk = i & 31;
+      const int t = t0 + row, e = e0 + row;
+      xs[kk][row] = t < T ? bf16_bits_to_float(x[(size_t)t * H + k0 + kk]) : 0.f;
+      ws[kk][row] = e < E ? Wr[(size_t)e * H + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = xs[kk][ty * 4 + i];
+        b[i] = ws[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
+    }
+  }
+}
+
+// Top-k per token (one warp per token): k rounds, each taking the largest
+// logit strictly below the previous winner in the order (logit desc, index
+// asc).  NaN logits rank as -inf.  Lane j keeps winner j; the weights are the
+// fp32 softmax over the winners.  Optionally marks the token in the expert's
+// membership bit map for the dispatch step.
+__global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                                   int32_t *__restrict__ idx, float *__restrict__ w,
+                                                   uint32_t *bitmap, int words) {
+  const int t = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float *row = logits + (size_t)t * E;
+  float lastv = INFINITY;
+  int laste = -1;
+  float myv = -INFINITY;
+  int mye = 0;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      float v = row[e];
+      if (v != v) v = -INFINITY;
+      const bool avail = (v < lastv) || (v == lastv && e > laste);
+      if (avail && (v > bv || (v == bv && e < be))) {
+        bv = v;
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    lastv = bv;
+    laste = be;
+    if (lane == r) {
+      myv = bv;
+      mye = be;
+    }
+  }
+  const float mx = __shfl_sync(0xffffffffu, myv, 0);
+  const float ex = lane < k ? expf(myv - mx) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = mye;
+    w[(size_t)t * k + lane] = ex / sum;
+    if (bitmap) atomicOr(&bitmap[(size_t)mye * words + (t >> 5)], 1u << (t & 31));
+  }
+}
+
+cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias, int T,
+                         const Workspace &ws, bool with_dispatch_bits, cudaStream_t s) {
+  const int H = d.hidden, E = d.n_experts, k = d.top_k;
+  if (T <= 8) {
+    trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
+    router_logits_small_kernel<<<(E + 3) / 4, 128, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin,
+                                                           ws.zero_words);
+    trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
+  } else {
+    dim3 grid((E + 63) / 64, (T + 63) / 64);
+    trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
+    router_logits_tiled_kernel<<<grid, 256, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin,
+                                                     ws.zero_words);
+    trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
+  }
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int blocks = (T * 32 + 255) / 256;
+  trace_mark(MOE_KERNEL_TOPK, false, s);
+  topk_kernel<<<blocks, 256, 0, s>>>(ws.logits, T, E, k, ws.idx, ws.w, with_dispatch_bits ? ws.bitmap : nullptr,
+                                     ws.words);
+  trace_mark(MOE_KERNEL_TOPK, true, s);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Dispatch: counts, offsets and a stable (expert, token)-ordered permutation.
+// The sorted position of slot (t, j) routed to expert e is
+//   offsets[e] + #{t' < t : t' routed to e},
+// read off the expert's membership bit map with popcounts, so the result is
+// independent of thread timing.  The shared expert's slots follow the routed
+// ones: position T*k + t.
+
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__restrict__ bitmap, int words, int E,
+                                                            int T, int k, uint32_t *__restrict__ wprefix,
+                                                            int32_t *counts, int32_t *offsets, int4 *items,
+                                                            uint32_t *n_items, uint32_t *done_counter) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (e < E) {
+    uint32_t run = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const int wi = w0 + lane;
+      const uint32_t bits = wi < words ? bitmap[(size_t)e * words + wi] : 0u;
+      const uint32_t cnt = __popc(bits);
+      uint32_t incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (wi < words) wprefix[(size_t)e * words + wi] = run + incl - cnt;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) counts[e] = (int32_t)run;
+  }
+  // The last block to finish turns counts into offsets and work items.
+  __shared__ bool is_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(done_counter, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  __shared__ int s_cnt[256], s_items[256];
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int eb = threadIdx.x * per, ee = min(E, eb + per);
+  int my_cnt = 0, my_items = 0;
+  for (int i = eb; i < ee; ++i) {
+    const int c = ((volatile int32_t *)counts)[i];
+    my_cnt += c;
+    my_items += (c + 7) >> 3;
+  }
+  s_cnt[threadIdx.x] = my_cnt;
+  s_items[threadIdx.x] = my_items;
+  __syncthreads();
+  if (threadIdx.x == 0) {  // tiny serial scan over 256 partial sums
+    int a = 0, b = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) {
+      const int ca = s_cnt[i], cb = s_items[i];
+      s_cnt[i] = a;
+      s_items[i] = b;
+      a += ca;
+      b += cb;
+    }
+    offsets[E] = a;  // == T * k
+    const int shared_items = (T + 7) >> 3;
+    for (int i = 0; i < shared_items; ++i)
+      items[b + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
+    *n_items = (uint32_t)(b + shared_items);
+  }
+  __syncthreads();
+  int pos = s_cnt[threadIdx.x], it = s_items[threadIdx.x];
+  for (int i = eb; i < ee; ++i) {
+    const int c = ((volatile int32_t *)counts)[i];
+    offsets[i] = pos;
+    for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
+    pos += c;
+  }
+}
+
+__global__ void dispatch_place_kernel(const int32_t *__restrict__ idx, const float *__restrict__ w, int T, int k,
+                                      int E, int words, const uint32_t *__restrict__ bitmap,
+                                      const uint32_t *__restrict__ wprefix, const int32_t *__restrict__ offsets,
+                                      int32_t *slot_pos, int32_t *sorted_tok, float *sorted_w, uint32_t *status) {
+  const long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long routed = (long long)T * k;
+  if (s >= routed + T) return;
+  if (s < routed) {
+    const int t = (int)(s / k);
+    const int e = idx[s];
+    if (e < 0 || e >= E) {
+      set_status(status, kStatusBadIndex);
+      slot_pos[s] = -1;  // the combine skips this slot
+      return;
+    }
+    const uint32_t word = bitmap[(size_t)e * words + (t >> 5)];
+    const int pos = offsets[e] + (int)wprefix[(size_t)e * words + (t >> 5)] + __popc(word & ((1u << (t & 31)) - 1u));
+    slot_pos[s] = pos;
+    sorted_tok[pos] = t;
+    sorted_w[pos] = w[s];
+  } else {
+    const int t = (int)(s - routed);
+    sorted_tok[routed + t] = t;
+    sorted_w[routed + t] = 1.f;
+  }
+}
+
+// Membership bits from a routing supplied by the caller (moe_experts_forward).
+__global__ void dispatch_bits_kernel(const int32_t *__restrict__ idx, int T, int k, int E, int words,
+                                     uint32_t *bitmap, uint32_t *status) {
+  const long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= (long long)T * k) return;
+  const int t = (int)(s / k);
+  const int e = idx[s];
+  if (e < 0 || e >= E) {
+    set_status(status, kStatusBadIndex);
+    return;
+  }
+  atomicOr(&bitmap[(size_t)e * words + (t >> 5)], 1u << (t & 31));
+}
+
+cudaError_t launch_dispatch_bits(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(ws.zero_begin, 0, ws.zero_words * 4, s);
+  if (err != cudaSuccess) return err;
+  const long long n = (long long)T * d.top_k;
+  trace_mark(MOE_KERNEL_DISPATCH_BITS, false, s);
+  dispatch_bits_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ws.idx, T, d.top_k, d.n_experts, ws.words,
+                                                                    ws.bitmap, ws.status);
+  trace_mark(MOE_KERNEL_DISPATCH_BITS, true, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s) {
+  const int E = d.n_experts, k = d.top_k;
+  trace_mark(MOE_KERNEL_DISPATCH_SCAN, false, s);
+  dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, s>>>(ws.bitmap, ws.words, E, T, k, ws.wprefix, ws.counts, ws.offsets,
+                                                   ws.items, ws.n_items, ws.done_counter);
+  trace_mark(MOE_KERNEL_DISPATCH_SCAN, true, s);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const long long n = (long long)T * k + T;
+  trace_mark(MOE_KERNEL_DISPATCH_PLACE, false, s);
+  dispatch_place_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ws.idx, ws.w, T, k, E, ws.words, ws.bitmap,
+                                                                     ws.wprefix, ws.offsets, ws.slot_pos,
+                                                                     ws.sorted_tok, ws.sorted_w, ws.status);
+  trace_mark(MOE_KERNEL_DISPATCH_PLACE, true, s);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Combine: out[t] = Y_shared[t] + sum_j w[t,j] Y[slot(t,j)], fp32 in a fixed
+// order (shared first, then j = 0..k-1), rounded once to bf16.
+__global__ void combine_kernel(const float *__restrict__ Y, const int32_t *__restrict__ slot_pos,
+                               const float *__restrict__ topk_w, int T, int k, int H, uint16_t *__restrict__ out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int per_row = H >> 2;
+  if (i >= (long long)T * per_row) return;
+  const int t = (int)(i / per_row), c4 = (int)(i % per_row);
+  float4 acc = reinterpret_cast<const float4 *>(Y + ((size_t)T * k + t) * H)[c4];
+  for (int j = 0; j < k; ++j) {
+    const int pos = slot_pos[(size_t)t * k + j];
+    if (pos < 0) continue;
+    const float wj = topk_w[(size_t)t * k + j];
+    const float4 v = reinterpret_cast<const float4 *>(Y + (size_t)pos * H)[c4];
+    acc.x = fmaf(wj, v.x, acc.x);
+    acc.y = fmaf(wj, v.y, acc.y);
+    acc.z = fmaf(wj, v.z, acc.z);
+    acc.w = fmaf(wj, v.w, acc.w);
+  }
+  uint2 o;
+  o.x = pack_bf16x2(acc.x, acc.y);
+  o.y = pack_bf16x2(acc.z, acc.w);
+  reinterpret_cast<uint2 *>(out + (size_t)t * H)[c4] = o;
+}
+
+cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s) {
+  const long long n = (long long)T * (d.hidden / 4);
+  trace_mark(MOE_KERNEL_COMBINE, false, s);
+  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ws.y, ws.slot_pos, ws.w, T, d.top_k, d.hidden, out);
+  trace_mark(MOE_KERNEL_COMBINE, true, s);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Between layers: resid += y (optional); x_norm = bf16(resid * rsqrt(mean(resid^2) + eps)).
+__global__ void __launch_bounds__(256) rmsnorm_residual_kernel(float *__restrict__ resid,
+                                                               const uint16_t *__restrict__ y,
+                                                               uint16_t *__restrict__ x_norm, int H, float eps) {
+  const int t = blockIdx.x;
+  float *r = resid + (size_t)t * H;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v = r[i];
+    if (y) {
+      v += bf16_bits_to_float(y[(size_t)t * H + i]);
+      r[i] = v;
+    }
+    ss = fmaf(v, v, ss);
+  }
+  __shared__ float part[32];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (threadIdx.x == 0) part[0] = v;
+  }
+  __syncthreads();
+  const float scale = 1.0f / sqrtf(part[0] / (float)H + eps);
+  for (int i = threadIdx.x; i < H; i += blockDim.x) x_norm[(size_t)t * H + i] = float_to_bf16_bits(r[i] * scale);
+}
+
+cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,
+                                    cudaStream_t s) {
+  rmsnorm_residual_kernel<<<T, 256, 0, s>>>(resid, y, x_norm, H, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

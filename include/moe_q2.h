@@ -1,0 +1,187 @@
+/*
+ * moe_q2.h -- C ABI of a B200 (sm_100a) library for one routed
+ * mixture-of-experts FFN layer whose experts are stored as 2-bit block
+ * ("Q2") quantized weights.
+ *
+ * The problem, as the pages state it: a sparse MoE model of 48 layers x 512
+ * routed experts in which every token is sent to 10 routed experts plus 1
+ * shared expert (Strata tuning page, section 2, model table; devlabs page,
+ * section 1 "MoE 专家分流"); the expert matmuls run directly from the
+ * quantized blocks, which are never densified at load (strata-mlx page, "它是
+ * 什么", first bullet); the 2-bit format decodes through an affine codebook
+ * with bias -1 (devlabs page, section 4, second validation layer).  Prompts
+ * arrive in 1024-token chunks (devlabs page, section 1) or larger chunks such
+ * as 32768 (Strata tuning page, section 4), decode/verify windows hold 1-3
+ * tokens (guess-and-check, devlabs page, section 1).
+ *
+ * Conventions for every call
+ *  - Every pointer is a DEVICE pointer unless the comment says otherwise.  The
+ *    caller allocates and owns all memory (weights, activations, outputs,
+ *    workspace); the library allocates nothing in these calls and keeps no
+ *    mutable global state (apart from the per-thread profiling switch
+ *    moe_trace_kernel), so calls on different streams with different
+ *    workspaces are independent.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  Argument checks run on the host before any
+ *    launch and return an error with nothing enqueued.
+ *  - Activations are bfloat16, passed as uint16_t bit patterns, row-major
+ *    [T, hidden].  Router weights are fp32 [n_experts, hidden] row-major.
+ *  - Kernels never trap or assert.  An inconsistency found on the device sets
+ *    a sticky status word in the workspace; moe_check_status() reads it.
+ */
+#ifndef MOE_Q2_H
+#define MOE_Q2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA headers. */
+struct CUstream_st;
+typedef struct CUstream_st *moe_stream_t;
+
+/* Layer dimensions.  The Q2 block is fixed at 32 weights.
+ * Limits checked by every call: hidden and inter are multiples of 128 in
+ * [128, 4096]; 1 <= n_experts <= 4096; 1 <= top_k <= min(n_experts, 32). */
+typedef struct {
+  int32_t hidden;    /* H: model width (router and expert input/output size) */
+  int32_t inter;     /* I: expert intermediate size (gate/up rows, down columns) */
+  int32_t n_experts; /* E: routed experts (the shared expert is separate) */
+  int32_t top_k;     /* k: routed experts per token */
+} moe_dims;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,         /* a size or pointer is invalid */
+  MOE_ERR_ALIGN = 2,       /* a pointer is not 16-byte aligned */
+  MOE_ERR_WORKSPACE = 3,   /* workspace smaller than moe_workspace_bytes() */
+  MOE_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+  MOE_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+  MOE_ERR_DEVICE = 6,      /* a kernel found an inconsistent index */
+  MOE_ERR_UNSUPPORTED = 7  /* not supported on this device (needs sm_100) */
+} moe_status;
+
+/* Router: w [n_experts, hidden] fp32; bias [n_experts] fp32 or NULL (no bias). */
+typedef struct {
+  const float *w;
+  const float *bias;
+} moe_router;
+
+/* Routed experts: n_experts packed experts back to back, stride moe_packed_expert_bytes(). */
+typedef struct {
+  const void *packed;
+} moe_experts;
+
+/* The shared expert: one packed expert, applied to every token with weight 1. */
+typedef struct {
+  const void *packed;
+} moe_shared;
+
+/* ---- Q2 weights ------------------------------------------------------------
+ * Canonical (input) format.  A block is 10 bytes: the fp16 scale d
+ * (little-endian), then 8 code bytes; element j (0..31) is the 2-bit code
+ * q = (code[j >> 2] >> (2*(j & 3))) & 3 and the weight is d * (q - 1)
+ * ("affine, bias = -1" codebook, devlabs page, section 4).  One expert is three
+ * row-major matrices back to back, blocks running along the contraction
+ * dimension: gate [inter x hidden/32 blocks], up [inter x hidden/32],
+ * down [hidden x inter/32].  moe_canonical_expert_bytes() gives its size.
+ *
+ * Packed format: the kernel layout written by moe_pack_q2; opaque to callers,
+ * same number of bytes as the canonical format, padded to 256 bytes per expert. */
+
+/* Host.  Bytes of one canonical expert (0 if dims are invalid). */
+size_t moe_canonical_expert_bytes(const moe_dims *dims);
+/* Host.  Bytes of one packed expert, the stride of moe_experts.packed (0 if invalid). */
+size_t moe_packed_expert_bytes(const moe_dims *dims);
+
+/* Repack n_experts canonical experts (device, back to back, stride
+ * moe_canonical_expert_bytes) into the kernel layout (device, stride
+ * moe_packed_expert_bytes).  packed_bytes is the size of the output buffer.
+ * Untimed set-up step; canonical and packed must not overlap. */
+moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_experts, void *packed,
+                       size_t packed_bytes, moe_stream_t stream);
+
+/* ---- workspace --------------------------------------------------------------
+ * Host.  Bytes of scratch memory moe_route / moe_layer_forward need for up to
+ * max_T tokens (0 if invalid).  One workspace must not be used by two calls
+ * that can run at the same time. */
+size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T);
+
+/* ---- routing ------------------------------------------------------------------
+ * For each of T tokens: logits[e] = sum_h x[h] Wr[e][h] + bias[e] (fp32
+ * accumulation); the top_k experts by logit, ties to the lower index, in
+ * descending-logit order; weights = softmax over the selected logits (fp32),
+ * which is the full softmax renormalised over the selected set.
+ * x [T, hidden] bf16; topk_idx [T, top_k] int32 and topk_w [T, top_k] fp32 are
+ * outputs.  T = 0 is a no-op. */
+moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_router *router, int32_t T,
+                     int32_t *topk_idx, float *topk_w, void *workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- the layer ------------------------------------------------------------------
+ * out[t] = shared(x[t]) + sum_j w[t,j] * expert_{idx[t,j]}(x[t]), with
+ * expert(v) = Wd (silu(Wg v) * (Wu v)) and silu(z) = z / (1 + exp(-z)).
+ * Rounding points: x is bf16; every dot product accumulates in fp32; the
+ * SwiGLU output h is rounded to bf16 before the down projection; the weighted
+ * sum is fp32 and out is rounded to bf16 (nearest even).
+ * x [T, hidden] bf16 in; out [T, hidden] bf16 out (must not overlap x).
+ * topk_idx_out [T, top_k] / topk_w_out [T, top_k]: optional copies of the
+ * routing decision (NULL to skip).  T = 0 is a no-op. */
+moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_router *router,
+                             const moe_experts *experts, const moe_shared *shared, uint16_t *out, int32_t T,
+                             int32_t *topk_idx_out, float *topk_w_out, void *workspace, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* The expert half of the layer for a routing decision made elsewhere:
+ * dispatch (per-expert counts, offsets, stable token permutation), the routed
+ * and shared SwiGLU experts and the weighted combine, with the rounding points
+ * of moe_layer_forward.  topk_idx [T, top_k] int32 (each in [0, n_experts),
+ * distinct per token) and topk_w [T, top_k] fp32 are inputs; an index out of
+ * range sets MOE_ERR_DEVICE in the workspace status and that slot is skipped.
+ * moe_layer_forward == moe_route followed by this call. */
+moe_status moe_experts_forward(const moe_dims *dims, const uint16_t *x, const int32_t *topk_idx,
+                               const float *topk_w, const moe_experts *experts, const moe_shared *shared,
+                               uint16_t *out, int32_t T, void *workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- between layers (a stack of layers) -------------------------------------------
+ * resid [T, hidden] fp32 (in/out), y [T, hidden] bf16 (may be NULL),
+ * x_norm [T, hidden] bf16 (out):
+ *   if y: resid += y;  then  x_norm = bf16(resid / sqrt(mean(resid^2) + eps)).
+ * Unit gain.  Used as x_{l+1} = x_l + MoE_l(RMSNorm(x_l)). */
+moe_status moe_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int32_t T, int32_t hidden,
+                                float eps, moe_stream_t stream);
+
+/* ---- profiling aid ------------------------------------------------------------------
+ * While kernel_id >= 0, every later call made by this host thread records the
+ * CUDA event `before` (a cudaEvent_t created by the caller) on its stream just
+ * before it launches kernel `kernel_id`, and `after` just after, as external
+ * event records, so they also become nodes of a CUDA graph being captured.
+ * kernel_id < 0 turns this off.  The setting is per host thread.  The kernel
+ * ids below name the library's kernels and may change between versions. */
+enum {
+  MOE_KERNEL_ROUTER_LOGITS = 0,
+  MOE_KERNEL_TOPK = 1,
+  MOE_KERNEL_DISPATCH_BITS = 2,
+  MOE_KERNEL_DISPATCH_SCAN = 3,
+  MOE_KERNEL_DISPATCH_PLACE = 4,
+  MOE_KERNEL_GATE_UP = 5,
+  MOE_KERNEL_DOWN = 6,
+  MOE_KERNEL_COMBINE = 7
+};
+moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after);
+
+/* ---- status ----------------------------------------------------------------------
+ * Blocking host call: waits for `stream`, reads and clears the sticky device
+ * status word in `workspace`; MOE_OK, MOE_ERR_DEVICE or MOE_ERR_TIMEOUT. */
+moe_status moe_check_status(void *workspace, moe_stream_t stream);
+
+/* Host.  Static string for a status code. */
+const char *moe_status_str(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_Q2_H */

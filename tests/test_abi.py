@@ -1,0 +1,81 @@
+"""The C-ABI library: it loads, exports every declared entry point, and its
+host-side checks reject bad arguments before touching a device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import __graft_entry__
+from bit_block_quantized_moe_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    __graft_entry__.build()
+    return B.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe_q2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(B.EXPORTED) == names
+
+
+def test_sizes(lib):
+    d = B.moe_dims(2048, 512, 512, 10)
+    assert B.moe_canonical_expert_bytes(d) == 983040
+    assert B.moe_packed_expert_bytes(d) == 983040
+    assert B.moe_workspace_bytes(d, 1024) > B.moe_workspace_bytes(d, 3) > 0
+    assert B.moe_workspace_bytes(d, -1) == 0
+
+
+@pytest.mark.parametrize("dims", [(2048, 512, 512, 0), (2048, 512, 512, 33), (2000, 512, 512, 10),
+                                  (2048, 500, 512, 10), (8192, 512, 512, 10), (256, 128, 4, 5),
+                                  (256, 128, 5000, 10)])
+def test_bad_dims_rejected(lib, dims):
+    d = B.moe_dims(*dims)
+    assert B.moe_packed_expert_bytes(d) == 0
+    assert B.moe_workspace_bytes(d, 8) == 0
+    r = B.moe_router(16, None)
+    ex, sh = B.moe_experts(16), B.moe_shared(16)
+    code = lib.moe_layer_forward(ctypes.byref(d), 16, ctypes.byref(r), ctypes.byref(ex), ctypes.byref(sh), 4096, 3,
+                                 None, None, 16, 1 << 30, None)
+    assert code == 1  # MOE_ERR_ARG
+
+
+def test_host_checks_before_launch(lib):
+    d = B.moe_dims(256, 128, 16, 2)
+    ws = B.moe_workspace_bytes(d, 8)
+    r = B.moe_router(0x1000, None)
+    ex, sh = B.moe_experts(0x2000), B.moe_shared(0x3000)
+
+    def call(x=0x4000, out=0x8000, T=8, wsp=0x10000, wsb=ws, rr=r):
+        return lib.moe_layer_forward(ctypes.byref(d), x, ctypes.byref(rr), ctypes.byref(ex), ctypes.byref(sh), out,
+                                     T, None, None, wsp, wsb, None)
+
+    assert call(T=0) == 0                      # T = 0: no-op, nothing launched
+    assert call(T=-1) == 1
+    assert call(x=0x4001) == 2                 # misaligned x
+    assert call(wsp=0x10008) == 2              # misaligned workspace
+    assert call(wsb=ws - 1) == 3               # workspace too small
+    assert call(out=0x4000 + 256) == 1         # out overlaps x
+    assert call(rr=B.moe_router(None, None)) == 1
+    assert lib.moe_check_status(None, None) == 1
+    assert B.moe_status_str(3) == "workspace too small"
+    assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, -1, 0x2000, 1 << 20, None) == 1
+    assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 0, 0x2000, 0, None) == 0
+    assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 2, 0x2000, 100, None) == 1    # output too small
+    assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 2, 0x2004, 1 << 20, None) == 2
+    assert lib.moe_rmsnorm_residual(None, None, None, 0, 256, 1e-6, None) == 0
+    assert lib.moe_rmsnorm_residual(None, None, None, 4, 256, 1e-6, None) == 1

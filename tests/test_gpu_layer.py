@@ -1,0 +1,173 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gen import CONFIGS, MoeConfig, make_x
+from parity import GAP_TIE, W_TOL, build_layer, check_layer, check_routing, gpu_forward, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    import __graft_entry__
+
+    __graft_entry__.build()
+    assert torch.cuda.is_available()
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return build_layer(CONFIGS[0])
+
+
+@pytest.fixture(scope="module")
+def full():
+    return build_layer(CONFIGS[2])  # full-size layer with the Zipf router bias
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 7, 8, 9, 33, 100, 257])
+def test_tiny_layer_all_tokens(tiny, T):
+    L, w = tiny
+    x = make_x(T, 256, seed=100 + T)
+    y, idx, wts = gpu_forward(L, x)
+    err, l2, flagged = check_layer(CONFIGS[0], w, x, y, idx, wts)
+    assert l2 < 5e-3
+
+
+def test_config0_exact_workload(tiny):
+    L, w = tiny
+    x = make_x(CONFIGS[0], seed=0)
+    y, idx, wts = gpu_forward(L, x)
+    check_layer(CONFIGS[0], w, x, y, idx, wts)
+
+
+@pytest.mark.parametrize("dims", [(384, 256, 8, 3), (256, 128, 1, 1), (256, 128, 16, 16), (128, 384, 32, 5),
+                                  (1024, 128, 64, 8)])
+def test_odd_shapes(dims):
+    H, I, E, k = dims
+    cfg = MoeConfig("t", H, I, E, k, 13, "zipf")
+    L, w = build_layer(cfg, seed=3)
+    for T in (1, 13):
+        x = make_x(T, H, seed=T)
+        y, idx, wts = gpu_forward(L, x)
+        check_layer(cfg, w, x, y, idx, wts)
+
+
+def test_decode_window_full_size(full):
+    L, w = full
+    cfg = CONFIGS[1]
+    for T in (1, 2, 3):
+        x = make_x(T, cfg.hidden, seed=7)
+        y, idx, wts = gpu_forward(L, x)
+        err, l2, flagged = check_layer(cfg, w, x, y, idx, wts)
+        print(f"T={T}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+
+
+def test_config1_uniform_router():
+    cfg = CONFIGS[1]
+    L, w = build_layer(cfg)
+    x = make_x(cfg, seed=0)
+    y, idx, wts = gpu_forward(L, x)
+    err, l2, flagged = check_layer(cfg, w, x, y, idx, wts)
+    print(f"config1: max-rel {err:.3e} relL2 {l2:.3e}")
+
+
+def test_config2_prefill_chunk(full):
+    cfg = CONFIGS[2]
+    L, w = full
+    x = make_x(cfg, seed=0)
+    y, idx, wts = gpu_forward(L, x)
+    # routing: every token against the oracle
+    idx_o, w_o, gap, _ = oracle.route(x, w["router_w"], w["router_b"], cfg.top_k)
+    flagged = check_routing(idx, wts, idx_o, w_o, gap)
+    # outputs: a seeded sample of tokens (and every flagged one)
+    rng = np.random.default_rng(0)
+    sample = np.union1d(rng.choice(cfg.tokens, 192, replace=False), np.array(flagged, dtype=np.int64))
+    sample = np.union1d(sample, [0, cfg.tokens - 1])
+    err, l2, _ = check_layer(cfg, w, x, y, idx, wts, tokens=sample)
+    print(f"config2: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+
+
+def test_prefill_ragged_and_cold_tail():
+    cfg = MoeConfig("cold", 2048, 512, 512, 10, 133, "zipf_cold")
+    L, w = build_layer(cfg, seed=1)
+    x = make_x(cfg, seed=1)
+    y, idx, wts = gpu_forward(L, x)
+    check_layer(cfg, w, x, y, idx, wts)
+
+
+def test_route_entry_point(full):
+    L, w = full
+    cfg = CONFIGS[2]
+    for T in (3, 1024):
+        x = make_x(T, cfg.hidden, seed=11)
+        idx, wts = L.route(to_dev_bf16(x))
+        torch.cuda.synchronize()
+        idx_o, w_o, gap, _ = oracle.route(x, w["router_w"], w["router_b"], cfg.top_k)
+        check_routing(idx.cpu().numpy(), wts.cpu().numpy(), idx_o, w_o, gap)
+
+
+def test_deterministic_and_zero_tokens(tiny):
+    L, w = tiny
+    x = make_x(100, 256, seed=5)
+    y1, i1, w1 = gpu_forward(L, x)
+    y2, i2, w2 = gpu_forward(L, x)
+    assert np.array_equal(y1, y2) and np.array_equal(i1, i2) and np.array_equal(w1, w2)
+    out = torch.full((1, 256), 7, dtype=torch.int16, device="cuda")
+    L.forward(torch.empty((0, 256), dtype=torch.int16, device="cuda"), out=out[:0])
+    torch.cuda.synchronize()
+    assert torch.all(out == 7)
+
+
+def test_rmsnorm_residual():
+    from bit_block_quantized_moe_b200 import moe_rmsnorm_residual
+
+    T, H = 37, 2048
+    rng = np.random.default_rng(0)
+    resid = rng.standard_normal((T, H)).astype(np.float32)
+    y = make_x(T, H, seed=9)
+    r_d = torch.from_numpy(resid.copy()).cuda()
+    y_d = to_dev_bf16(y)
+    xn = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    moe_rmsnorm_residual(r_d, y_d, xn, T, H, 1e-6)
+    torch.cuda.synchronize()
+    r_ref = resid.astype(np.float64) + (y.astype(np.uint32) << 16).view(np.float32)
+    assert np.max(np.abs(r_d.cpu().numpy() - r_ref)) < 1e-5
+    want = oracle.rmsnorm(r_ref, 1e-6)
+    got = (xn.cpu().numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    assert np.max(np.abs(got - want) / np.maximum(np.abs(want), 1e-3)) < 2 ** -8
+
+
+def test_experts_forward_given_routing(tiny):
+    L, w = tiny
+    cfg = CONFIGS[0]
+    T = 21
+    x = make_x(T, 256, seed=3)
+    rng = np.random.default_rng(0)
+    forced = np.stack([rng.choice(16, 2, replace=False) for _ in range(T)]).astype(np.int32)
+    y_o, _, w_o, _ = oracle.layer(x, w["router_w"], w["router_b"], w["experts"], w["shared"], 2, 128,
+                                  forced_idx=forced)
+    out = L.experts_forward(to_dev_bf16(x), torch.from_numpy(forced).cuda(),
+                            torch.from_numpy(w_o.astype(np.float32)).cuda())
+    torch.cuda.synchronize()
+    L.check_status()
+    y = (out.cpu().numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    assert np.max(np.abs(y - y_o)) / np.max(np.abs(y_o)) <= 1e-2
+
+
+def test_experts_forward_bad_index_sets_status(tiny):
+    from bit_block_quantized_moe_b200 import MoeError
+
+    L, w = tiny
+    T = 4
+    x = make_x(T, 256, seed=4)
+    idx = torch.tensor([[0, 1], [2, 99], [3, 4], [-5, 6]], dtype=torch.int32, device="cuda")
+    wt = torch.full((T, 2), 0.5, dtype=torch.float32, device="cuda")
+    L.experts_forward(to_dev_bf16(x), idx, wt)
+    with pytest.raises(MoeError) as ei:
+        L.check_status()
+    assert ei.value.code == 6  # MOE_ERR_DEVICE
+    L.check_status()  # cleared
