@@ -52,6 +52,9 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_items = take((size_t)max_items * 16);
   const size_t o_h = take(slots * I * 2);
   const size_t o_y = take(slots * H * 4);
+  const bool fused = decode_fused_supported(d, T);
+  const size_t o_tcnt = take(fused ? decode_counter_words(d) * 4 : 0);
+  const size_t o_part = take(fused ? decode_partial_floats(d, T) * 4 : 0);
   if (base && ws) {
     uint8_t *b = static_cast<uint8_t *>(base);
     ws->status = reinterpret_cast<uint32_t *>(b + o_hdr);
@@ -72,6 +75,9 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->items = reinterpret_cast<int4 *>(b + o_items);
     ws->h = reinterpret_cast<uint16_t *>(b + o_h);
     ws->y = reinterpret_cast<float *>(b + o_y);
+    ws->gbar = reinterpret_cast<uint32_t *>(b + o_hdr + 64);
+    ws->tile_cnt = reinterpret_cast<uint32_t *>(b + o_tcnt);
+    ws->partial = reinterpret_cast<float *>(b + o_part);
     ws->words = (int)words;
     ws->max_items = max_items;
   }
@@ -114,7 +120,13 @@ size_t moe_packed_expert_bytes(const moe_dims *dims) {
 
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T) {
   if (!dims_ok(dims) || max_T < 0) return 0;
-  return workspace_layout(*dims, max_T, nullptr, nullptr);
+  // enough for every T <= max_T (the small-T layout carries the fused-decode regions)
+  size_t need = workspace_layout(*dims, max_T, nullptr, nullptr);
+  for (int t = 1; t <= 8 && t <= max_T; ++t) {
+    const size_t n = workspace_layout(*dims, t, nullptr, nullptr);
+    need = n > need ? n : need;
+  }
+  return need;
 }
 
 moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_experts, void *packed,
@@ -195,6 +207,12 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
   workspace_layout(*dims, T, workspace, &ws);
   if (topk_idx_out) ws.idx = topk_idx_out;
   if (topk_w_out) ws.w = topk_w_out;
+  if (decode_fused_supported(*dims, T)) {
+    return cuda_status(launch_decode_fused(*dims, x, router->w, router->bias,
+                                           static_cast<const uint8_t *>(experts->packed),
+                                           static_cast<const uint8_t *>(shared->packed), T, ws, topk_idx_out,
+                                           topk_w_out, out, s));
+  }
   cudaError_t err = launch_route(*dims, x, router->w, router->bias, T, ws, true, s);
   if (err == cudaSuccess) err = run_experts(*dims, x, experts, shared, out, T, ws, s, true);
   return cuda_status(err);

@@ -64,10 +64,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---- Q2 fragment decode ----------------------------------------------------------
-// One 32-bit code word holds 8 pairs; pair p keeps its even-k code at bits 2p and
-// its odd-k code at bits 16+2p.  OR-ing the masked code into the mantissa of
-// bf16 128.0 gives 128 + q*4^s exactly (s = 0,1,2); one bf16x2 FMA then yields
-// q - 1 exactly.
+// A packed 32-bit code word holds the 16 codes one lane needs for the two
+// m16n8k16 steps of a 32-weight block: 8 pairs, the even-k code of a pair in
+// the low half-word and the odd-k code at the same offset in the high half.
+// Pair (step s, fragment register P) sits at bit 8s + {0, 4, 2, 6}[P], so that
+// P0/P1 (k pair 4c, 4c+1) are read with the mask 0x3 and P2/P3 (k pair 4c+2,
+// 4c+3) with the mask 0xC after shifts of 0, 4, 8, 12.  OR-ing a masked code
+// into the mantissa of bf16 128.0 gives 128 + q (mask 0x3) or 128 + 4q (mask
+// 0xC), exactly.
+// Bit offset of fragment register P (0..3) in step 0.
+__host__ __device__ constexpr int pair_pos(int P) { return P == 0 ? 0 : (P == 1 ? 4 : (P == 2 ? 2 : 6)); }
+
+// Biased decode: p[0..3] / p[4..7] are the A registers of steps 0 / 1 holding
+// 128 + q (P0, P1) and 128 + 4q (P2, P3).  Used with the B registers of P2/P3
+// scaled by 1/4 and the accumulator started at -sum_k c_k x_k with c_k = 129
+// (k % 4 < 2) or 33 (k % 4 >= 2), which leaves sum_k (q_k - 1) x_k.
+__device__ __forceinline__ void decode_q2_biased(uint32_t w, uint32_t (&p)[8]) {
+  constexpr uint32_t kMagic = 0x43004300u;  // bf16 pair (128, 128)
+  const uint32_t w4 = w >> 4, w8 = w >> 8, w12 = w >> 12;
+  p[0] = (w & 0x00030003u) | kMagic;
+  p[1] = (w4 & 0x00030003u) | kMagic;
+  p[2] = (w & 0x000C000Cu) | kMagic;
+  p[3] = (w4 & 0x000C000Cu) | kMagic;
+  p[4] = (w8 & 0x00030003u) | kMagic;
+  p[5] = (w12 & 0x00030003u) | kMagic;
+  p[6] = (w8 & 0x000C000Cu) | kMagic;
+  p[7] = (w12 & 0x000C000Cu) | kMagic;
+}
 
 __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
@@ -75,43 +98,35 @@ __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t 
   return d;
 }
 
-// Decodes the 8 pairs of `w` into q-1 as bf16x2 (exact).
-__device__ __forceinline__ void decode_q2_word(uint32_t w, uint32_t (&p)[8]) {
-  constexpr uint32_t kMagic = 0x43004300u;  // (128, 128)
-  constexpr uint32_t kOne = 0x3F803F80u;    // (1, 1)
-  constexpr uint32_t kQuarter = 0x3E803E80u;
-  constexpr uint32_t kSixteenth = 0x3D803D80u;
-  constexpr uint32_t kM129 = 0xC301C301u;   // (-129, -129)
-  constexpr uint32_t kM33 = 0xC204C204u;    // (-33, -33)
-  constexpr uint32_t kM9 = 0xC110C110u;     // (-9, -9)
-  uint32_t w6 = w >> 6, w12 = w >> 12;
-  p[0] = bf16x2_fma((w & 0x00030003u) | kMagic, kOne, kM129);
-  p[1] = bf16x2_fma((w & 0x000C000Cu) | kMagic, kQuarter, kM33);
-  p[2] = bf16x2_fma((w & 0x00300030u) | kMagic, kSixteenth, kM9);
-  p[3] = bf16x2_fma((w6 & 0x00030003u) | kMagic, kOne, kM129);
-  p[4] = bf16x2_fma((w6 & 0x000C000Cu) | kMagic, kQuarter, kM33);
-  p[5] = bf16x2_fma((w6 & 0x00300030u) | kMagic, kSixteenth, kM9);
-  p[6] = bf16x2_fma((w12 & 0x00030003u) | kMagic, kOne, kM129);
-  p[7] = bf16x2_fma((w12 & 0x000C000Cu) | kMagic, kQuarter, kM33);
+// Exact decode: the same registers holding q - 1 (one bf16x2 FMA per pair, exact).
+__device__ __forceinline__ void decode_q2_exact(uint32_t w, uint32_t (&p)[8]) {
+  constexpr uint32_t kOne = 0x3F803F80u;      // (1, 1)
+  constexpr uint32_t kQuarter = 0x3E803E80u;  // (1/4, 1/4)
+  constexpr uint32_t kM129 = 0xC301C301u;     // (-129, -129)
+  constexpr uint32_t kM33 = 0xC204C204u;      // (-33, -33)
+  decode_q2_biased(w, p);
+  p[0] = bf16x2_fma(p[0], kOne, kM129);
+  p[1] = bf16x2_fma(p[1], kOne, kM129);
+  p[2] = bf16x2_fma(p[2], kQuarter, kM33);
+  p[3] = bf16x2_fma(p[3], kQuarter, kM33);
+  p[4] = bf16x2_fma(p[4], kOne, kM129);
+  p[5] = bf16x2_fma(p[5], kOne, kM129);
+  p[6] = bf16x2_fma(p[6], kQuarter, kM33);
+  p[7] = bf16x2_fma(p[7], kQuarter, kM33);
 }
 
 // D = A(16x16 bf16) * B(16x8 bf16) + C, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
                                                const float (&c)[4]) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%10,%11,%12,%13};\n"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
+// Read-only global load through the non-coherent path (weights, router).
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
 __device__ __forceinline__ void set_status(uint32_t *status, uint32_t bit) {
   if (status) atomicOr(status, bit);

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(256) expert_mma_kernel(ExpertArgs a) {
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
           uint32_t p[8];
-          decode_q2_word(cws[blk], p);
+          decode_q2_exact(cws[blk], p);
           const int kb = 128 * grp + 32 * blk;
           const uint2 b0 = *reinterpret_cast<const uint2 *>(xrow + kb);
           const uint2 b1 = *reinterpret_cast<const uint2 *>(xrow + kb + 16);

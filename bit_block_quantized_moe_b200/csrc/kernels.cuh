@@ -25,6 +25,9 @@ struct Workspace {
   int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)
   uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position
   float *y;                // [T*k + T][H] fp32 expert outputs by sorted position
+  uint32_t *gbar;          // grid barrier of the fused decode kernel: count, generation (kept zeroed)
+  uint32_t *tile_cnt;      // fused decode: per-tile arrival counters, then per-expert ready counters
+  float *partial;          // fused decode: per (expert, tile) partial outputs
   int words;               // ceil(T / 32)
   int max_items;
 };
@@ -43,6 +46,12 @@ cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaS
 cudaError_t launch_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                            const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s);
+bool decode_fused_supported(const moe_dims &d, int T);
+size_t decode_partial_floats(const moe_dims &d, int T);
+size_t decode_counter_words(const moe_dims &d);
+cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias,
+                                const uint8_t *experts, const uint8_t *shared, int T, const Workspace &ws,
+                                int32_t *idx_out, float *w_out, uint16_t *out, cudaStream_t s);
 cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,
                                     cudaStream_t s);
 

@@ -8,6 +8,7 @@
 #include <float.h>
 
 #include "kernels.cuh"
+#include "router.cuh"
 
 namespace moe {
 
@@ -20,10 +21,11 @@ namespace moe {
 // (128 weights); a group stores 32 lanes x 16 bytes of codes followed by
 // 8 x 16 bytes of scales.  Lane (g = lane/4, c = lane%4) owns tile rows g and
 // g+8; its word for block b holds, for k16 step s in {0,1}, the k pairs
-// (4c, 4c+1) and (4c+2, 4c+3) of both rows: pair p = 4s + P with
+// (4c, 4c+1) and (4c+2, 4c+3) of both rows, one pair per A-fragment register P:
 // P = 0: row g, k 4c;  P = 1: row g+8, k 4c;  P = 2: row g, k 4c+2;  P = 3: row g+8, k 4c+2
-// (k relative to 32b + 16s); the even-k code sits at bit 2p, the odd-k code
-// at bit 16+2p.  Scales: for g in 0..7, block 0..3: (d[row g], d[row g+8]).
+// (k relative to 32b + 16s); the even-k code sits at bit 8s + {0,4,2,6}[P],
+// the odd-k code 16 bits higher.  Scales: for g in 0..7, block 0..3:
+// (d[row g], d[row g+8]).
 __global__ void pack_q2_kernel(const uint8_t *__restrict__ canon, uint8_t *__restrict__ packed, int n_experts,
                                PackedGeom G, size_t canon_stride) {
   const int ug_per_expert = G.gu_units * G.gu_groups + G.dn_units * G.dn_groups;
@@ -76,8 +78,9 @@ __global__ void pack_q2_kernel(const uint8_t *__restrict__ canon, uint8_t *__res
       const int s = p >> 2, P = p & 3;
       const int rho = g + 8 * (P & 1);
       const int k = 32 * b + 16 * s + 4 * c + 2 * (P >> 1);
-      w |= code(rho, k) << (2 * p);
-      w |= code(rho, k + 1) << (16 + 2 * p);
+      const int pos = 8 * s + pair_pos(P);
+      w |= code(rho, k) << pos;
+      w |= code(rho, k + 1) << (16 + pos);
     }
     words[wi] = w;
   }
@@ -116,49 +119,25 @@ __device__ __forceinline__ void clear_range(uint32_t *p, size_t n) {
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
 }
 
-// Few tokens (T <= 8): one warp per expert row, 128-bit streaming loads of Wr.
+// Few tokens (T <= 8): one CTA of 4 warps per expert row, warp q summing the
+// row's quarter q (router_quarter), combined in quarter order.
 __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t *__restrict__ x,
                                                                    const float *__restrict__ Wr,
                                                                    const float *__restrict__ bias, int T, int H,
                                                                    int E, float *__restrict__ logits,
                                                                    uint32_t *zero_p, size_t zero_n) {
   clear_range(zero_p, zero_n);
+  __shared__ float part[8][4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (e >= E) return;
-  const float *wrow = Wr + (size_t)e * H;
+  const int e = blockIdx.x;
   float acc[8];
-#pragma unroll
-  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-#pragma unroll 4
-  for (int k = lane * 4; k < H; k += 128) {
-    const uint4 wv = ldg_nc_v4(wrow + k);
-    const float w0 = __uint_as_float(wv.x), w1 = __uint_as_float(wv.y), w2 = __uint_as_float(wv.z),
-                w3 = __uint_as_float(wv.w);
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      if (t < T) {
-        const uint2 xv = *reinterpret_cast<const uint2 *>(x + (size_t)t * H + k);
-        float a = acc[t];
-        a = fmaf(__uint_as_float(xv.x << 16), w0, a);
-        a = fmaf(__uint_as_float(xv.x & 0xffff0000u), w1, a);
-        a = fmaf(__uint_as_float(xv.y << 16), w2, a);
-        a = fmaf(__uint_as_float(xv.y & 0xffff0000u), w3, a);
-        acc[t] = a;
-      }
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-  }
+  router_quarter<false>(x, H, T, Wr + (size_t)e * H, H, warp, lane, acc);
   if (lane == 0) {
-    const float b = bias ? bias[e] : 0.f;
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
-      if (t < T) logits[(size_t)t * E + e] = acc[t] + b;
+    for (int t = 0; t < 8; ++t) part[t][warp] = acc[t];
   }
+  __syncthreads();
+  if (threadIdx.x < T) logits[(size_t)threadIdx.x * E + e] = router_combine(part[threadIdx.x], bias ? bias[e] : 0.f);
 }
 
 // Many tokens: 64 tokens x 64 experts per CTA, fp32 FMA tiles through shared memory.
@@ -208,59 +187,28 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(const uint16_t
   }
 }
 
-// Top-k per token (one warp per token): k rounds, each taking the largest
-// logit strictly below the previous winner in the order (logit desc, index
-// asc).  NaN logits rank as -inf.  Lane j keeps winner j; the weights are the
-// fp32 softmax over the winners.  Optionally marks the token in the expert's
-// membership bit map for the dispatch step.
+// Top-k per token, one warp per token (see warp_topk); optionally marks the
+// token in the expert's membership bit map for the dispatch step.
 __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int T, int E, int k,
                                                    int32_t *__restrict__ idx, float *__restrict__ w,
                                                    uint32_t *bitmap, int words) {
+  __shared__ uint64_t scratch[8][64];
   const int t = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
+  float wt;
+  int e;
   const float *row = logits + (size_t)t * E;
-  float lastv = INFINITY;
-  int laste = -1;
-  float myv = -INFINITY;
-  int mye = 0;
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      float v = row[e];
-      if (v != v) v = -INFINITY;
-      const bool avail = (v < lastv) || (v == lastv && e > laste);
-      if (avail && (v > bv || (v == bv && e < be))) {
-        bv = v;
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    lastv = bv;
-    laste = be;
-    if (lane == r) {
-      myv = bv;
-      mye = be;
-    }
-  }
-  const float mx = __shfl_sync(0xffffffffu, myv, 0);
-  const float ex = lane < k ? expf(myv - mx) : 0.f;
-  float sum = ex;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (E <= 512)
+    warp_topk_fast<16>(row, E, k, lane, scratch[threadIdx.x >> 5], e, wt);
+  else if (E <= 1024)
+    warp_topk_fast<32>(row, E, k, lane, scratch[threadIdx.x >> 5], e, wt);
+  else
+    warp_topk(row, E, k, lane, e, wt);
   if (lane < k) {
-    idx[(size_t)t * k + lane] = mye;
-    w[(size_t)t * k + lane] = ex / sum;
-    if (bitmap) atomicOr(&bitmap[(size_t)mye * words + (t >> 5)], 1u << (t & 31));
+    idx[(size_t)t * k + lane] = e;
+    w[(size_t)t * k + lane] = wt;
+    if (bitmap) atomicOr(&bitmap[(size_t)e * words + (t >> 5)], 1u << (t & 31));
   }
 }
 
@@ -269,8 +217,7 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, 
   const int H = d.hidden, E = d.n_experts, k = d.top_k;
   if (T <= 8) {
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
-    router_logits_small_kernel<<<(E + 3) / 4, 128, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin,
-                                                           ws.zero_words);
+    router_logits_small_kernel<<<E, 128, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin, ws.zero_words);
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
   } else {
     dim3 grid((E + 63) / 64, (T + 63) / 64);

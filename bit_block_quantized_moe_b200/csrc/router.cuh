@@ -1,0 +1,213 @@
+// Router arithmetic shared by the stand-alone routing kernels and the fused
+// decode kernel, so that both take bit-identical routing decisions.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Router arithmetic for T <= 8 tokens.  The row is cut into 4 quarters of
+// H/4; quarter q is summed by one warp: lane l accumulates k = q*H/4 + 4l +
+// 128 i in order, then a butterfly sum.  The logit is ((p0 + p1) + p2) + p3 + b.
+// Both the routing kernel and the fused decode kernel use exactly this order,
+// so they take identical routing decisions.
+template <bool kWrShared>
+__device__ __forceinline__ void router_quarter(const uint16_t *x, int xstride, int T, const float *wrow, int H,
+                                               int quarter, int lane, float (&acc)[8]) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+  const int kq = H / 4;
+#pragma unroll 4
+  for (int k = quarter * kq + lane * 4; k < (quarter + 1) * kq; k += 128) {
+    const uint4 wv = kWrShared ? *reinterpret_cast<const uint4 *>(wrow + k) : ldg_nc_v4(wrow + k);
+    const float w0 = __uint_as_float(wv.x), w1 = __uint_as_float(wv.y), w2 = __uint_as_float(wv.z),
+                w3 = __uint_as_float(wv.w);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (t < T) {
+        const uint2 xv = *reinterpret_cast<const uint2 *>(x + (size_t)t * xstride + k);
+        float a = acc[t];
+        a = fmaf(__uint_as_float(xv.x << 16), w0, a);
+        a = fmaf(__uint_as_float(xv.x & 0xffff0000u), w1, a);
+        a = fmaf(__uint_as_float(xv.y << 16), w2, a);
+        a = fmaf(__uint_as_float(xv.y & 0xffff0000u), w3, a);
+        acc[t] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+  }
+}
+
+__device__ __forceinline__ float router_combine(const float *part4, float b) {
+  return ((part4[0] + part4[1]) + part4[2]) + part4[3] + b;
+}
+
+// fp32 softmax over the k winners held by lanes 0..k-1 (lane order = selection order).
+__device__ __forceinline__ float topk_softmax(float myv, int lane, int k) {
+  const float mx = __shfl_sync(0xffffffffu, myv, 0);
+  const float ex = lane < k ? expf(myv - mx) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  return ex / sum;
+}
+
+// Warp arg-max of (value desc, index asc) over the lanes' candidates.
+__device__ __forceinline__ void warp_argmax(float &bv, int &be) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+    if (ov > bv || (ov == bv && oe < be)) {
+      bv = ov;
+      be = oe;
+    }
+  }
+}
+
+// Top-k with the token's logits held in registers (E <= 32 * NPL): one read
+// of the row, then k selection rounds in registers.  Same selection rule and
+// softmax as warp_topk, hence the same result.
+template <int NPL>
+__device__ __forceinline__ void warp_topk_regs(const float *row, int E, int k, int lane, int &e_out, float &w_out) {
+  float v[NPL];
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    const int e = lane + 32 * j;
+    float t = e < E ? __ldcg(row + e) : -INFINITY;
+    if (t != t) t = -INFINITY;
+    v[j] = t;
+  }
+  float lastv = INFINITY;
+  int laste = -1;
+  float myv = -INFINITY;
+  int mye = 0;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      const int e = lane + 32 * j;  // increasing in j: the first of equal values has the lower index
+      const float t = v[j];
+      const bool avail = e < E && ((t < lastv) || (t == lastv && e > laste));
+      if (avail && (be == 0x7fffffff || t > bv)) {
+        bv = t;
+        be = e;
+      }
+    }
+    warp_argmax(bv, be);
+    lastv = bv;
+    laste = be;
+    if (lane == r) {
+      myv = bv;
+      mye = be;
+    }
+  }
+  e_out = mye;
+  w_out = topk_softmax(myv, lane, k);
+}
+
+// Top-k of one token's logits (one warp): k rounds, each taking the largest
+// logit strictly after the previous winner in the order (logit desc, index
+// asc); NaN ranks as -inf.  Lane j < k returns winner j (e) and its weight,
+// the fp32 softmax over the k winners.  Logits are read through L2 (.cg) so
+// values written by other CTAs of the same kernel are seen.
+__device__ __forceinline__ void warp_topk(const float *row, int E, int k, int lane, int &e_out, float &w_out) {
+  float lastv = INFINITY;
+  int laste = -1;
+  float myv = -INFINITY;
+  int mye = 0;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      float v = __ldcg(row + e);
+      if (v != v) v = -INFINITY;
+      const bool avail = (v < lastv) || (v == lastv && e > laste);
+      if (avail && (v > bv || (v == bv && e < be))) {
+        bv = v;
+        be = e;
+      }
+    }
+    warp_argmax(bv, be);
+    lastv = bv;
+    laste = be;
+    if (lane == r) {
+      myv = bv;
+      mye = be;
+    }
+  }
+  e_out = mye;
+  w_out = topk_softmax(myv, lane, k);
+}
+
+// Monotonic 32-bit key of a float (larger float -> larger key); NaN ranks as -inf.
+__device__ __forceinline__ uint32_t float_key(float v) {
+  if (v != v) v = -INFINITY;
+  if (v == 0.f) v = 0.f;  // -0 and +0 are equal logits (the index decides)
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Top-k by threshold, filter and rank (E <= 32 * NPL, one warp).  Each
+// (logit, index) becomes a 64-bit value key << 32 | ~index, so that "larger"
+// is the selection order (logit desc, index asc).  The k-th largest of the 32
+// lane maxima bounds the k-th largest overall from below; the values at or
+// above it (usually a few more than k) are compacted one per lane and ranked
+// by counting.  Falls back to warp_topk_regs when more than 32 values pass.
+// `scratch` is 64 uint64 of shared memory private to the warp.  Same
+// selection and softmax as warp_topk, hence the same result.
+template <int NPL>
+__device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, int lane, uint64_t *scratch,
+                                               int &e_out, float &w_out) {
+  uint64_t v[NPL];
+  uint64_t m = 0;
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = e < E ? ((uint64_t)float_key(__ldcg(row + e)) << 32) | (uint32_t)~e : 0ull;
+    m = v[j] > m ? v[j] : m;
+  }
+  int rank = 0;
+#pragma unroll 8
+  for (int o = 0; o < 32; ++o) rank += __shfl_sync(0xffffffffu, m, o) > m;
+  const uint32_t sel = __ballot_sync(0xffffffffu, rank == k - 1);
+  const uint64_t L = __shfl_sync(0xffffffffu, m, __ffs(sel) - 1);
+  int cnt = 0;
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) cnt += v[j] >= L;
+  const int total = __reduce_add_sync(0xffffffffu, cnt);
+  if (total > 32) {
+    __syncwarp();
+    warp_topk_regs<NPL>(row, E, k, lane, e_out, w_out);
+    return;
+  }
+  int base = 0;
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    const bool p = v[j] >= L;
+    const uint32_t bal = __ballot_sync(0xffffffffu, p);
+    if (p) scratch[base + __popc(bal & ((1u << lane) - 1u))] = v[j];
+    base += __popc(bal);
+  }
+  __syncwarp();
+  const uint64_t cand = lane < total ? scratch[lane] : 0ull;
+  int r = 0;
+  for (int o = 0; o < total; ++o) r += scratch[o] > cand;
+  __syncwarp();
+  if (lane < total && r < k) scratch[32 + r] = cand;
+  __syncwarp();
+  const uint64_t mine = lane < k ? scratch[32 + lane] : 0ull;
+  __syncwarp();
+  e_out = (int)~(uint32_t)mine;
+  w_out = topk_softmax(key_float((uint32_t)(mine >> 32)), lane, k);
+}
+
+}  // namespace moe

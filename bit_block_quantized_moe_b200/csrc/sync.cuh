@@ -1,0 +1,130 @@
+// Device-side synchronisation primitives with bounded waits (sm_100a).
+//
+// Every wait here gives up after kWaitLimitNs of %globaltimer time, reports
+// the timeout through the caller's status word and returns false, so that no
+// kernel can spin forever.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---- mbarrier ------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete; false after the limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+// ---- bulk copies (TMA engine, no tensor map) ---------------------------------------
+// global -> shared, completion counted in bytes on `bar`.  16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ---- CTA-level ---------------------------------------------------------------------
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
+
+// ---- grid-level ----------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Loads through L2 only (data written earlier in the same kernel by other CTAs).
+__device__ __forceinline__ uint2 ldg_cg_v2(const void *p) { return __ldcg(reinterpret_cast<const uint2 *>(p)); }
+__device__ __forceinline__ float4 ldg_cg_f4(const void *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
+
+// Grid-wide barrier for a co-resident (cooperatively launched) grid.  The
+// participating threads of each CTA first meet at named barrier `bar_id`;
+// thread `leader` arrives on the global counter; the last CTA to arrive resets
+// the counter and bumps the generation word the others wait on.  Leaves
+// count == 0, so the next barrier (or the next launch) starts clean.
+// Returns false (and sets the status timeout bit) if the wait hit the limit.
+__device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t *gen, int bar_id, int nthreads, bool leader,
+                                             uint32_t *status, int *flag_smem) {
+  named_bar(bar_id, nthreads);
+  if (leader) {
+    bool ok = true;
+    const uint32_t g = ld_acquire_gpu(gen);
+    __threadfence();
+    const uint32_t arrived = atomicAdd(count, 1u) + 1u;
+    if (arrived == gridDim.x) {
+      atomicExch(count, 0u);
+      __threadfence();
+      st_release_gpu(gen, g + 1u);
+    } else {
+      const uint64_t t0 = global_timer_ns();
+      while (ld_acquire_gpu(gen) == g) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          set_status(status, kStatusTimeout);
+          ok = false;
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    *flag_smem = ok ? 0 : 1;
+  }
+  named_bar(bar_id, nthreads);
+  return *(volatile int *)flag_smem == 0;
+}
+
+}  // namespace moe

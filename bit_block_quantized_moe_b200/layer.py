@@ -50,7 +50,7 @@ class Q2MoeLayer:
     def reserve(self, T: int):
         if T > self._ws_T:
             nbytes = B.moe_workspace_bytes(self.dims, T)
-            self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
             self._ws_T = T
 
     def forward(self, x, out=None, topk_idx=None, topk_w=None, stream=None):

@@ -105,9 +105,11 @@ moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_ex
                        size_t packed_bytes, moe_stream_t stream);
 
 /* ---- workspace --------------------------------------------------------------
- * Host.  Bytes of scratch memory moe_route / moe_layer_forward need for up to
- * max_T tokens (0 if invalid).  One workspace must not be used by two calls
- * that can run at the same time. */
+ * Host.  Bytes of scratch memory moe_route / moe_layer_forward /
+ * moe_experts_forward need for up to max_T tokens (0 if invalid).  Its first
+ * 4 bytes hold the sticky device status word: zero the workspace (or at least
+ * those 4 bytes) once after allocating it.  One workspace must not be used by
+ * two calls that can run at the same time. */
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T);
 
 /* ---- routing ------------------------------------------------------------------
@@ -168,7 +170,8 @@ enum {
   MOE_KERNEL_DISPATCH_PLACE = 4,
   MOE_KERNEL_GATE_UP = 5,
   MOE_KERNEL_DOWN = 6,
-  MOE_KERNEL_COMBINE = 7
+  MOE_KERNEL_COMBINE = 7,
+  MOE_KERNEL_DECODE_FUSED = 8
 };
 moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after);
 

@@ -171,3 +171,29 @@ def test_experts_forward_bad_index_sets_status(tiny):
         L.check_status()
     assert ei.value.code == 6  # MOE_ERR_DEVICE
     L.check_status()  # cleared
+
+
+@pytest.mark.parametrize("T", [4, 5, 8])
+def test_fused_decode_window_sizes(full, T):
+    L, w = full
+    x = make_x(T, 2048, seed=40 + T)
+    y, idx, wts = gpu_forward(L, x)
+    err, l2, flagged = check_layer(CONFIGS[2], w, x, y, idx, wts)
+    print(f"fused T={T}: max-rel {err:.3e} relL2 {l2:.3e}")
+
+
+def test_fused_decode_agrees_with_route_and_general_path(full):
+    L, w = full
+    T = 3
+    x = make_x(T, 2048, seed=77)
+    xd = to_dev_bf16(x)
+    y1, idx1, w1 = gpu_forward(L, x)
+    y2, idx2, w2 = gpu_forward(L, x)
+    assert np.array_equal(y1, y2) and np.array_equal(idx1, idx2)  # deterministic
+    ridx, rw = L.route(xd)
+    torch.cuda.synchronize()
+    assert np.array_equal(ridx.cpu().numpy(), idx1) and np.array_equal(rw.cpu().numpy(), w1)
+    out = L.experts_forward(xd, ridx, rw)  # general dispatch path, same routing
+    torch.cuda.synchronize()
+    yg = (out.cpu().numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    assert np.max(np.abs(yg - y1)) <= 4e-3 * np.max(np.abs(y1))
