@@ -1,5 +1,5 @@
 // Fused decode/verify-window layer (T <= 8 tokens) in one persistent,
-// cooperatively launched kernel (sm_100a).  One CTA per SM: 16 consumer
+// cooperatively launched kernel (sm_100a).  One CTA per SM: 14 consumer
 // warps and 1 producer warp.
 //
 //  A  The producer bulk-copies (TMA engine) the tokens and this CTA's router
@@ -13,15 +13,17 @@
 //  C  Work lists, expert-major, cut into equal contiguous ranges per CTA:
 //     gate/up units (expert, 8 intermediate rows) and down pairs (expert, 16
 //     output rows).  The producer streams the CTA's units into a ring of
-//     shared-memory stages as stages free up.  Gate/up: K split over the 16
-//     warps, partial sums reduced through a double-buffered shared slot by a
-//     rotating epilogue warp (mbarrier hand-off, no CTA-wide barrier), which
-//     writes h = silu(g) * u (bf16).  At the end the CTA publishes, per
-//     expert, how many of its units are done.
-//  D  Down pairs, 4 warps per pair (K split), once the expert's h is
-//     complete (per-expert counter, bounded wait): partial = w[t, e] * (Wd_e
-//     h_e) per (expert, tile).  The last CTA to contribute to a tile sums its
-//     partials in expert order and writes out (bf16).
+//     shared-memory stages as stages free up; stage s belongs to consumer
+//     warp s % 14, which computes the whole unit (full K) with no cross-warp
+//     reduction and writes h = silu(g) * u (bf16) straight from its
+//     accumulators.  At the end the CTA publishes, per expert, how many of
+//     its units are done.
+//  D  Once the h of the (at most two) experts in the CTA's down range is
+//     complete (per-expert counter, bounded wait) it is copied into shared
+//     memory; each down stage (up to 4 pairs) again belongs to one warp:
+//     partial = w[t, e] * (Wd_e h_e) per (expert, tile).  The last CTA to
+//     contribute to a tile sums its partials in expert order and writes out
+//     (bf16).
 // Dequantisation happens in registers and feeds m16n8k16 tensor-core MMAs
 // with the tokens as the 8 columns; gate/up uses the biased decode with the
 // -1 offset folded into the accumulator start (decode_q2_biased), down the
@@ -34,16 +36,15 @@ namespace moe {
 
 namespace {
 
-constexpr int kConsumerWarps = 16;
+constexpr int kConsumerWarps = 14;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kMaxTok = 8;
 constexpr int kMaxSel = 128;              // T * top_k
 constexpr int kMaxEntries = kMaxSel + 1;  // touched experts + shared
 constexpr int kMaxE = 1024;
-constexpr int kNR = 2;                    // gate/up reduction slots
-constexpr int kBarConsumers = 1;          // named barrier ids (0 = __syncthreads)
-constexpr int kBarPairLane0 = 2;          // 2..5
+constexpr int kMaxI = 512;                // down K handled by the h cache
+constexpr int kBarConsumers = 1;          // named barrier id (0 = __syncthreads)
 
 struct DecodeArgs {
   const uint16_t *x;
@@ -75,16 +76,16 @@ __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v
 __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes) {
   SmemLayout L;
   uint32_t o = 0;
-  L.bars = o;  // full[ns], empty[ns], rbar, xbar, rfull[kNR], rfree[kNR]
-  o = align_to(o + 8u * (2 * ns + 2 + 2 * kNR), 16);
+  L.bars = o;  // full[ns], empty[ns], rbar, xbar
+  o = align_to(o + 8u * (2 * ns + 2), 16);
   L.xs = o;
   o = align_to(o + (uint32_t)T * (H + 16) * 2, 16);
   L.corr = o;
   o = align_to(o + (uint32_t)(H / 32) * kMaxTok * 4, 16);
-  L.rpart = o;  // [4 rows][8 tokens][4 quarters]
+  L.rpart = o;  // [rows per pass <= 4][8 tokens][4 quarters]
   o += 4 * kMaxTok * 4 * 4;
-  L.red = o;    // gate/up: [kNR][16 warps][32][4]; down: [2][4 lanes][4][32][4]; top-k scratch
-  o += kNR * kConsumerWarps * 32 * 16;
+  L.red = o;    // top-k scratch (phase B), then the h cache of phase D: [2 entries][8 tokens][I + 16]
+  o += align_to(2u * kMaxTok * (kMaxI + 16) * 2, 16);
   L.sel_idx = o;
   o += kMaxSel * 4;
   L.sel_w = o;
@@ -109,7 +110,6 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
 // B-operand scale 1/4 for the fragment registers of k pair (4c+2, 4c+3); exact.
 __device__ __forceinline__ uint32_t bf16x2_quarter(uint32_t v) { return bf16x2_fma(v, 0x3E803E80u, 0x80008000u); }
 
-template <int GPW>  // gate/up block groups per consumer warp (H / 128 / 16)
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const PackedGeom &G = a.G;
@@ -119,8 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   uint64_t *empty = full + a.ns;
   uint64_t *rbar = empty + a.ns;
   uint64_t *xbar = rbar + 1;
-  uint64_t *rfull = xbar + 1;
-  uint64_t *rfree = rfull + kNR;
   uint16_t *xs = reinterpret_cast<uint16_t *>(smem + L.xs);
   float *corr = reinterpret_cast<float *>(smem + L.corr);
   float *rpart = reinterpret_cast<float *>(smem + L.rpart);
@@ -158,14 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   if (tid == 0) {
     for (int i = 0; i < a.ns; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kConsumerWarps);
+      mbar_init(&empty[i], 1);  // each stage is consumed by one warp
     }
     mbar_init(rbar, 1);
     mbar_init(xbar, 1);
-    for (int i = 0; i < kNR; ++i) {
-      mbar_init(&rfull[i], kConsumerWarps);
-      mbar_init(&rfree[i], 1);
-    }
     mbar_fence_init();
     for (int i = 0; i < 8; ++i) misc[i] = 0;
   }
@@ -212,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       corr[b * kMaxTok + t] = s;
     }
     bounded_wait(rbar, 0);
-    for (int r0 = 0; r0 < n_rrows; r0 += 4) {
+    constexpr int kRowsPerPass = kConsumerWarps / 4;  // 4 warps (quarters) per router row
+    for (int r0 = 0; r0 < n_rrows; r0 += kRowsPerPass) {
       const int r = r0 + (warp >> 2), q = warp & 3;
       if (r < n_rrows) {
         float acc[8];
@@ -223,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         }
       }
       named_bar(kBarConsumers, kConsumers);
-      if (tid < 4 * T) {
+      if (tid < kRowsPerPass * T) {
         const int rr = tid / T, t = tid % T;
         if (r0 + rr < n_rrows) {
           const int e = blockIdx.x + gridDim.x * (r0 + rr);
@@ -349,88 +344,74 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   }
 
   // ---------------- consumers, phase C: gate/up + SwiGLU ----------------
-  const int kw = warp;  // K split over the 16 consumer warps
-  uint32_t B[GPW][4][2][2];
-  float negC[GPW][4][2];
-#pragma unroll
-  for (int gi = 0; gi < GPW; ++gi)
-#pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-      const int b = (kw * GPW + gi) * 4 + blk;
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        uint2 v = make_uint2(0u, 0u);
-        if (g < T) v = *reinterpret_cast<const uint2 *>(xs + g * xstride + 32 * b + 16 * s + 4 * c);
-        B[gi][blk][s][0] = v.x;
-        B[gi][blk][s][1] = bf16x2_quarter(v.y);
-      }
-      negC[gi][blk][0] = 2 * c < T ? -corr[b * kMaxTok + 2 * c] : 0.f;
-      negC[gi][blk][1] = 2 * c + 1 < T ? -corr[b * kMaxTok + 2 * c + 1] : 0.f;
-    }
+  // B fragments read the tokens from shared memory: scale the k pair (4c+2,
+  // 4c+3) of every 4 by 1/4 in place (exact) and negate the correction sums.
+  for (int i = tid; i < T * (H / 4); i += kConsumers) {
+    uint32_t *p2 = reinterpret_cast<uint32_t *>(xs + (i / (H / 4)) * xstride + 4 * (i % (H / 4)) + 2);
+    *p2 = bf16x2_quarter(*p2);
+  }
+  for (int i = tid; i < (H / 32) * kMaxTok; i += kConsumers) corr[i] = (i % kMaxTok) < T ? -corr[i] : 0.f;
+  named_bar(kBarConsumers, kConsumers);
 
-  int s_idx = 0;
-  for (; s_idx < n_gu_st; ++s_idx) {
+  const uint16_t *xrow = xs + (g < T ? g : 0) * xstride + 4 * c;
+  const bool row_ok = g < T;
+  for (int s_idx = warp; s_idx < n_gu_st; s_idx += kConsumerWarps) {
     const int slot = s_idx % a.ns;
     bounded_wait(&full[slot], (s_idx / a.ns) & 1);
     const uint8_t *st = ring + (size_t)slot * a.stage_bytes;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int gi = 0; gi < GPW; ++gi) {
-      const uint8_t *gp = st + (size_t)(kw * GPW + gi) * kGroupBytes;
+    for (int grp = 0; grp < G.gu_groups; ++grp) {
+      // one block group: 4 independent block tiles, staged load -> decode -> MMA -> scale
+      const uint8_t *gp = st + (size_t)grp * kGroupBytes;
       const uint4 cw = lds128(gp + lane * 16);
       const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
       const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
       const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+      uint2 b0[4], b1[4];
+      float2 nc[4];
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
-        uint32_t p[8];
-        decode_q2_biased(cws[blk], p);
-        const uint32_t a0[4] = {p[0], p[1], p[2], p[3]};
-        const uint32_t a1[4] = {p[4], p[5], p[6], p[7]};
-        const float cin[4] = {negC[gi][blk][0], negC[gi][blk][1], negC[gi][blk][0], negC[gi][blk][1]};
-        float d[4];
-        mma_bf16_16816(d, a0, B[gi][blk][0][0], B[gi][blk][0][1], cin);
-        mma_bf16_16816(d, a1, B[gi][blk][1][0], B[gi][blk][1][1], d);
+        const int b = grp * 4 + blk;
+        b0[blk] = *reinterpret_cast<const uint2 *>(xrow + 32 * b);
+        b1[blk] = *reinterpret_cast<const uint2 *>(xrow + 32 * b + 16);
+        if (!row_ok) b0[blk] = b1[blk] = make_uint2(0u, 0u);
+        nc[blk] = *reinterpret_cast<const float2 *>(corr + b * kMaxTok + 2 * c);
+      }
+      uint32_t p[4][8];
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) decode_q2_biased(cws[blk], p[blk]);
+      float d[4][4];
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        const uint32_t a0[4] = {p[blk][0], p[blk][1], p[blk][2], p[blk][3]};
+        const float cin[4] = {nc[blk].x, nc[blk].y, nc[blk].x, nc[blk].y};
+        mma_bf16_16816(d[blk], a0, b0[blk].x, b0[blk].y, cin);
+      }
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        const uint32_t a1[4] = {p[blk][4], p[blk][5], p[blk][6], p[blk][7]};
+        mma_bf16_16816(d[blk], a1, b1[blk].x, b1[blk].y, d[blk]);
+      }
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
         const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
-        acc[0] = fmaf(s2.x, d[0], acc[0]);
-        acc[1] = fmaf(s2.x, d[1], acc[1]);
-        acc[2] = fmaf(s2.y, d[2], acc[2]);
-        acc[3] = fmaf(s2.y, d[3], acc[3]);
+        acc[0] = fmaf(s2.x, d[blk][0], acc[0]);
+        acc[1] = fmaf(s2.x, d[blk][1], acc[1]);
+        acc[2] = fmaf(s2.y, d[blk][2], acc[2]);
+        acc[3] = fmaf(s2.y, d[blk][3], acc[3]);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
-    const int rs = s_idx % kNR, use = s_idx / kNR;
-    if (use > 0) bounded_wait(&rfree[rs], (use - 1) & 1);  // epilogue of unit s_idx - kNR done
-    float *rb = red + rs * (kConsumerWarps * 32 * 4);
-    *reinterpret_cast<float4 *>(rb + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&rfull[rs]);
-    if (warp == s_idx % kConsumerWarps) {
-      // epilogue for this unit: sum the 16 partials (warp order), SwiGLU, store h
-      bounded_wait(&rfull[rs], use & 1);
-      float sm[4] = {0.f, 0.f, 0.f, 0.f};
+    const int id = g0 + s_idx;
+    const int entry = id / G.gu_units, u = id % G.gu_units;
+    const int i = 8 * u + g;  // tile rows g (gate) and g+8 (up) share intermediate row i
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float4 v = *reinterpret_cast<const float4 *>(rb + (w * 32 + lane) * 4);
-        sm[0] += v.x;
-        sm[1] += v.y;
-        sm[2] += v.z;
-        sm[3] += v.w;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&rfree[rs]);
-      const int id = g0 + s_idx;
-      const int entry = id / G.gu_units, u = id % G.gu_units;
-      const int i = 8 * u + g;  // tile rows g (gate) and g+8 (up) share intermediate row i
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int n = 2 * c + half;
-        if (n < T) {
-          const int j = tokj[entry * kMaxTok + n];
-          if (j >= 0)
-            a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(sm[half]) * sm[2 + half]);
-        }
+    for (int half = 0; half < 2; ++half) {
+      const int n = 2 * c + half;
+      if (n < T) {
+        const int j = tokj[entry * kMaxTok + n];
+        if (j >= 0) a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(acc[half]) * acc[2 + half]);
       }
     }
   }
@@ -446,82 +427,84 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   }
 
   // ---------------- consumers, phase D: down projection + combine ----------------
-  const int pl = warp >> 2, kd = warp & 3;  // pair lane (0..3), K group (I / 128 == 4)
-  int cur_entry = -1;
-  uint32_t Bd[4][2][2];
-  int dbuf = 0;
-  for (int sd = 0; s_idx < n_st; ++s_idx, ++sd) {
+  // h of the experts in this CTA's down range (at most two) into shared memory.
+  uint16_t *hc = reinterpret_cast<uint16_t *>(red);
+  const int hstride = I + 16;
+  const int e_lo = d1 > d0 ? d0 / G.dn_units : 0;
+  const int n_hc = d1 > d0 ? (d1 - 1) / G.dn_units - e_lo + 1 : 0;
+  if (tid < n_hc && !*reinterpret_cast<volatile int *>(&misc[1])) {
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu(&ready[e_lo + tid]) < (uint32_t)G.gu_units) {
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        set_status(a.status, kStatusTimeout);
+        misc[1] = 1;
+        break;
+      }
+    }
+  }
+  named_bar(kBarConsumers, kConsumers);
+  for (int i = tid; i < n_hc * kMaxTok * (I / 8); i += kConsumers) {
+    const int he = i / (kMaxTok * (I / 8)), r = i % (kMaxTok * (I / 8));
+    const int t = r / (I / 8), c8 = r % (I / 8);
+    const int j = t < T ? tokj[(e_lo + he) * kMaxTok + t] : -1;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (j >= 0) v = __ldcg(reinterpret_cast<const uint4 *>(a.h + ((size_t)t * (K + 1) + j) * I + c8 * 8));
+    *reinterpret_cast<uint4 *>(hc + (he * kMaxTok + t) * hstride + c8 * 8) = v;
+  }
+  named_bar(kBarConsumers, kConsumers);
+
+  for (int s_idx = n_gu_st + ((warp - n_gu_st % kConsumerWarps + kConsumerWarps) % kConsumerWarps); s_idx < n_st;
+       s_idx += kConsumerWarps) {
+    const int sd = s_idx - n_gu_st;
     const int slot = s_idx % a.ns;
     bounded_wait(&full[slot], (s_idx / a.ns) & 1);
     const uint8_t *st = ring + (size_t)slot * a.stage_bytes;
     const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
-    for (int q = q0 + pl; q < q1; q += 4) {
+    for (int q = q0; q < q1; ++q) {
       const int entry = q / G.dn_units, tile = q % G.dn_units;
-      if (entry != cur_entry) {
-        cur_entry = entry;
-        // wait until every gate/up unit of this expert is published
-        if (lane == 0 && !*reinterpret_cast<volatile int *>(&misc[1])) {
-          const uint64_t t0 = global_timer_ns();
-          while (ld_acquire_gpu(&ready[entry]) < (uint32_t)G.gu_units) {
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-              set_status(a.status, kStatusTimeout);
-              misc[1] = 1;
-              break;
-            }
-          }
-        }
-        __syncwarp();
-        const int j = g < T ? tokj[entry * kMaxTok + g] : -1;
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk)
-#pragma unroll
-          for (int s = 0; s < 2; ++s) {
-            uint2 v = make_uint2(0u, 0u);
-            if (j >= 0) v = ldg_cg_v2(a.h + ((size_t)g * (K + 1) + j) * I + 128 * kd + 32 * blk + 16 * s + 4 * c);
-            Bd[blk][s][0] = v.x;
-            Bd[blk][s][1] = v.y;
-          }
-      }
-      const uint8_t *gp = st + (size_t)(q - q0) * G.dn_unit_bytes + (size_t)kd * kGroupBytes;
-      const uint4 cw = lds128(gp + lane * 16);
-      const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
-      const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
-      const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+      const uint16_t *hrow = hc + ((entry - e_lo) * kMaxTok + g) * hstride + 4 * c;
+      const uint8_t *pp_st = st + (size_t)(q - q0) * G.dn_unit_bytes;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int grp = 0; grp < 4; ++grp) {
+        const uint8_t *gp = pp_st + (size_t)grp * kGroupBytes;
+        const uint4 cw = lds128(gp + lane * 16);
+        const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
+        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+        const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+        uint2 b0[4], b1[4];
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        uint32_t p[8];
-        decode_q2_exact(cws[blk], p);
-        const uint32_t a0[4] = {p[0], p[1], p[2], p[3]};
-        const uint32_t a1[4] = {p[4], p[5], p[6], p[7]};
-        const float z[4] = {0.f, 0.f, 0.f, 0.f};
-        float d[4];
-        mma_bf16_16816(d, a0, Bd[blk][0][0], Bd[blk][0][1], z);
-        mma_bf16_16816(d, a1, Bd[blk][1][0], Bd[blk][1][1], d);
-        const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
-        acc[0] = fmaf(s2.x, d[0], acc[0]);
-        acc[1] = fmaf(s2.x, d[1], acc[1]);
-        acc[2] = fmaf(s2.y, d[2], acc[2]);
-        acc[3] = fmaf(s2.y, d[3], acc[3]);
-      }
-      float *rb = red + ((dbuf * 4 + pl) * 4) * 32 * 4;
-      *reinterpret_cast<float4 *>(rb + (kd * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      named_bar(kBarPairLane0 + pl, 128);
-      if (kd == 0) {
-        float sm[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float4 v = *reinterpret_cast<const float4 *>(rb + (w * 32 + lane) * 4);
-          sm[0] += v.x;
-          sm[1] += v.y;
-          sm[2] += v.z;
-          sm[3] += v.w;
+        for (int blk = 0; blk < 4; ++blk) {
+          const int b = grp * 4 + blk;
+          b0[blk] = *reinterpret_cast<const uint2 *>(hrow + 32 * b);
+          b1[blk] = *reinterpret_cast<const uint2 *>(hrow + 32 * b + 16);
         }
-        const float w0 = tokw[entry * kMaxTok + 2 * c], w1 = tokw[entry * kMaxTok + 2 * c + 1];
-        float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
-        *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(sm[0] * w0, sm[1] * w1, sm[2] * w0, sm[3] * w1);
+        uint32_t p[4][8];
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) decode_q2_exact(cws[blk], p[blk]);
+        float d[4][4];
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          const uint32_t a0[4] = {p[blk][0], p[blk][1], p[blk][2], p[blk][3]};
+          const float z[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16_16816(d[blk], a0, b0[blk].x, b0[blk].y, z);
+        }
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          const uint32_t a1[4] = {p[blk][4], p[blk][5], p[blk][6], p[blk][7]};
+          mma_bf16_16816(d[blk], a1, b1[blk].x, b1[blk].y, d[blk]);
+        }
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
+          acc[0] = fmaf(s2.x, d[blk][0], acc[0]);
+          acc[1] = fmaf(s2.x, d[blk][1], acc[1]);
+          acc[2] = fmaf(s2.y, d[blk][2], acc[2]);
+          acc[3] = fmaf(s2.y, d[blk][3], acc[3]);
+        }
       }
-      dbuf ^= 1;
+      const float w0 = tokw[entry * kMaxTok + 2 * c], w1 = tokw[entry * kMaxTok + 2 * c + 1];
+      float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
+      *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
@@ -530,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   // Count this CTA's contributions per output tile (one fence per writer
   // warp); the last contributor of a tile sums its partials in expert order.
   int *done_tiles = sel_idx;  // phase-B scratch, free now
-  if (kd == 0) __threadfence();
+  __threadfence();
   named_bar(kBarConsumers, kConsumers);
   for (int i = tid; i < d1 - d0; i += kConsumers) {
     const int tile = (d0 + i) % G.dn_units;
@@ -582,8 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
 bool decode_fused_supported(const moe_dims &d, int T) {
   const PackedGeom G = packed_geom(d.hidden, d.inter);
   if (T < 1 || T > kMaxTok || T * d.top_k > kMaxSel || d.n_experts > kMaxE) return false;
-  if (G.dn_groups != 4) return false;                         // down: 4 warps x 1 group (inter 512)
-  if (G.gu_groups != 16 && G.gu_groups != 32) return false;  // gate/up: 16 warps x 1 or 2 groups
+  if (G.dn_groups != 4) return false;  // down: 4 groups of 128 (inter 512, the h cache size)
   return true;
 }
 
@@ -639,12 +621,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   a.ns = ns;
   a.stage_bytes = stage_bytes;
 
-  void (*kern)(DecodeArgs) = nullptr;
-  switch (G.gu_groups / 16) {
-    case 1: kern = decode_fused_kernel<1>; break;
-    case 2: kern = decode_fused_kernel<2>; break;
-    default: return cudaErrorInvalidValue;
-  }
+  void (*kern)(DecodeArgs) = decode_fused_kernel;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (err != cudaSuccess) return err;
   int per_sm = 0;
