@@ -18,10 +18,10 @@ static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-static int max_items_for(const moe_dims &d, int T) {
+static int max_items_for(const moe_dims &d, int T, int tile) {
   const long long routed = (long long)T * d.top_k;
   const long long touched = routed < d.n_experts ? routed : d.n_experts;
-  return (int)(touched + (routed + 7) / 8 + (T + 7) / 8);
+  return (int)(touched + (routed + tile - 1) / tile + (T + tile - 1) / tile);
 }
 
 // Lays out the workspace for T tokens; returns the bytes needed.  With base ==
@@ -48,8 +48,11 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_slot = take((size_t)T * k * 4);
   const size_t o_stok = take(slots * 4);
   const size_t o_sw = take(slots * 4);
-  const int max_items = max_items_for(d, T);
+  const int max_items = max_items_for(d, T, 8);
   const size_t o_items = take((size_t)max_items * 16);
+  const int max_tc_items = max_items_for(d, T, 128);
+  const size_t o_tc_items = take((size_t)max_tc_items * 16);
+  const size_t o_xs = take(T > 8 ? slots * H * 2 : 0);
   const size_t o_h = take(slots * I * 2);
   const size_t o_y = take(slots * H * 4);
   const bool fused = decode_fused_supported(d, T);
@@ -73,6 +76,10 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->sorted_tok = reinterpret_cast<int32_t *>(b + o_stok);
     ws->sorted_w = reinterpret_cast<float *>(b + o_sw);
     ws->items = reinterpret_cast<int4 *>(b + o_items);
+    ws->tc_items = reinterpret_cast<int4 *>(b + o_tc_items);
+    ws->n_tc_items = reinterpret_cast<uint32_t *>(b + o_hdr + 8);
+    ws->xs = reinterpret_cast<uint16_t *>(b + o_xs);
+    ws->max_tc_items = max_tc_items;
     ws->h = reinterpret_cast<uint16_t *>(b + o_h);
     ws->y = reinterpret_cast<float *>(b + o_y);
     ws->gbar = reinterpret_cast<uint32_t *>(b + o_hdr + 64);
@@ -184,9 +191,12 @@ static cudaError_t run_experts(const moe_dims &d, const uint16_t *x, const moe_e
   cudaError_t err = cudaSuccess;
   if (!bits_ready) err = launch_dispatch_bits(d, T, ws, s);
   if (err == cudaSuccess) err = launch_dispatch(d, T, ws, s);
-  if (err == cudaSuccess)
-    err = launch_experts(d, G, static_cast<const uint8_t *>(experts->packed),
-                         static_cast<const uint8_t *>(shared->packed), x, T, ws, s);
+  if (err == cudaSuccess) {
+    const uint8_t *ex = static_cast<const uint8_t *>(experts->packed);
+    const uint8_t *sh = static_cast<const uint8_t *>(shared->packed);
+    // few tokens: register-dequant tensor-core tiles of 8 tokens; otherwise tcgen05 grouped GEMM
+    err = T <= 8 ? launch_experts(d, G, ex, sh, x, T, ws, s) : launch_tc_experts(d, G, ex, sh, x, T, ws, s);
+  }
   if (err == cudaSuccess) err = launch_combine(d, T, ws, out, s);
   return err;
 }

@@ -23,6 +23,9 @@ struct Workspace {
   int32_t *sorted_tok;     // [T*k + T]: token of each sorted position (shared slots last)
   float *sorted_w;         // [T*k + T]
   int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)
+  int4 *tc_items;          // [max_tc_items]: (expert, first position, tokens <= 128, 0)
+  uint32_t *n_tc_items;
+  uint16_t *xs;            // [T*k + T][H] bf16 token rows in sorted-position order
   uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position
   float *y;                // [T*k + T][H] fp32 expert outputs by sorted position
   uint32_t *gbar;          // grid barrier of the fused decode kernel: count, generation (kept zeroed)
@@ -30,6 +33,7 @@ struct Workspace {
   float *partial;          // fused decode: per (expert, tile) partial outputs
   int words;               // ceil(T / 32)
   int max_items;
+  int max_tc_items;
 };
 
 // Profiling hook (moe_trace_kernel): records the caller's events around kernel `id`.
@@ -45,6 +49,8 @@ cudaError_t launch_dispatch_bits(const moe_dims &d, int T, const Workspace &ws, 
 cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                            const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
+cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
+                              const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s);
 bool decode_fused_supported(const moe_dims &d, int T);
 size_t decode_partial_floats(const moe_dims &d, int T);

@@ -1,0 +1,355 @@
+// Grouped expert GEMMs for prefill chunks on the 5th-generation tensor cores
+// (tcgen05, sm_100a).
+//
+// One persistent CTA per SM walks a list of work items (expert, 128-row M
+// tile, up to 128 tokens).  For each 128-wide K chunk:
+//   producer warp   : bulk-copies the tile's packed Q2 codes + scales (8 units
+//                     x 640 B) and TMA-loads the chunk of the expert's token
+//                     rows (slot-sorted activations, 128-byte swizzle) into a
+//                     shared-memory stage;
+//   8 dequant warps : decode the codes in registers to bf16 d * (q - 1) and
+//                     store them into a tensor-memory A stage (tcgen05.st);
+//   MMA warp        : 8 x tcgen05.mma (A from tensor memory, B from shared
+//                     memory), fp32 accumulators in tensor memory, commits
+//                     release the stages;
+//   4 epilogue warps: tcgen05.ld the accumulators; gate/up writes
+//                     h = silu(g) * u (bf16), down writes the fp32 expert
+//                     output rows for the combine.
+// Accumulators are double-buffered so the epilogue of one item overlaps the
+// MMAs of the next.  Every wait is bounded (sync.cuh).
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "tc.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kStages = 4;         // shared-memory stages (A codes + B rows)
+constexpr int kAStages = 4;        // tensor-memory A stages
+constexpr int kTileUnits = 8;      // 16-row units per 128-row M tile
+constexpr int kABytes = kTileUnits * kGroupBytes;  // 5120
+constexpr int kBBox = 2048;        // one TMA box: 16 rows x 128 bytes
+constexpr int kBSub = 8 * kBBox;   // one 64-wide K half of the chunk, 128 rows: 16 KB
+constexpr int kStageBytes = 1024 * ((kABytes + 2 * kBSub + 1023) / 1024);  // 37888
+constexpr int kWarpProducer = 0, kWarpMMA = 1, kWarpDequant0 = 2, kNumDequant = 8, kWarpEpi0 = 10, kNumEpi = 4;
+constexpr int kThreadsTC = (kWarpEpi0 + kNumEpi) * 32;  // 448
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemA0 = 256;  // A stages live at columns 256 + 64 * sa; D buffers at 0 and 128
+
+struct TcArgs {
+  const uint8_t *experts;
+  const uint8_t *shared;
+  PackedGeom G;
+  int E;
+  const int4 *items;          // (expert or E for shared, first sorted position, tokens <= 128, 0)
+  const uint32_t *n_items;
+  int mtiles;                 // 128-row tiles per expert for this projection
+  int kchunks;                // 128-wide K chunks (block groups)
+  size_t unit_bytes;
+  size_t sec_off;             // section offset inside a packed expert
+  uint16_t *h_out;            // gate/up output [positions][I]
+  float *y_out;               // down output [positions][H]
+  uint32_t *status;
+};
+
+struct Bars {
+  uint64_t full[kStages], empty[kStages], afull[kAStages], aempty[kAStages], dfull[2], dempty[2], done;
+  uint32_t tmem;
+  int abort;
+};
+
+__device__ __forceinline__ bool waitb(uint64_t *bar, uint32_t parity, Bars &B, uint32_t *status) {
+  if (*reinterpret_cast<volatile int *>(&B.abort)) return false;
+  if (!mbar_wait(bar, parity)) {
+    set_status(status, kStatusTimeout);
+    B.abort = 1;
+    return false;
+  }
+  return true;
+}
+
+// Scales pair (d_g, d_g8) fp16 -> bf16 pairs (d, d) for the two rows.
+__device__ __forceinline__ void scale_pairs(uint32_t sh2, uint32_t &sg, uint32_t &sg8) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&sh2));
+  sg = pack_bf16x2(f.x, f.x);
+  sg8 = pack_bf16x2(f.y, f.y);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+template <int MODE>  // 0: gate/up + SwiGLU -> h (bf16); 1: down -> y (fp32)
+__global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  Bars &B = *reinterpret_cast<Bars *>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = (int)*a.n_items;
+  const int n_work = n_items * a.mtiles;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&B.full[i], 1);
+      mbar_init(&B.empty[i], kNumDequant + 1);  // dequant warps read A, the MMA commit releases B
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&B.afull[i], kNumDequant);
+      mbar_init(&B.aempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.dfull[i], 1);
+      mbar_init(&B.dempty[i], kNumEpi);
+    }
+    mbar_init(&B.done, 1);
+    B.abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == kWarpProducer) tmem_alloc(&B.tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = B.tmem;
+
+  if (warp == kWarpProducer) {
+    if (lane == 0) {
+      int cnt = 0;
+      for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+        const int4 it = a.items[w / a.mtiles];
+        const int mt = w % a.mtiles;
+        const int nb = (it.z + 15) >> 4;  // 16-row boxes
+        const uint8_t *ex = it.x == a.E ? a.shared : a.experts + (size_t)it.x * a.G.expert_bytes;
+        const uint8_t *abase = ex + a.sec_off + (size_t)mt * kTileUnits * a.unit_bytes;
+        for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
+          const int s = cnt % kStages;
+          if (!waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) continue;
+          uint8_t *st = smem + s * kStageBytes;
+          mbar_arrive_expect_tx(&B.full[s], (uint32_t)(kABytes + nb * 2 * kBBox));
+          for (int u = 0; u < kTileUnits; ++u)
+            bulk_g2s(st + u * kGroupBytes, abase + (size_t)u * a.unit_bytes + (size_t)kc * kGroupBytes, kGroupBytes,
+                     &B.full[s]);
+          uint8_t *bst = st + kABytes + (1024 - kABytes % 1024) % 1024;
+          for (int sub = 0; sub < 2; ++sub)
+            for (int b = 0; b < nb; ++b)
+              tma_load_2d(bst + sub * kBSub + b * kBBox, &tmB, kc * 128 + sub * 64, it.y + 16 * b, &B.full[s]);
+        }
+      }
+      // every copy issued must land before the CTA exits
+      for (int c2 = max(0, cnt - kStages); c2 < cnt; ++c2) waitb(&B.full[c2 % kStages], (c2 / kStages) & 1, B, a.status);
+    }
+  } else if (warp == kWarpMMA) {
+    if (lane == 0) {
+      int cnt = 0, acnt = 0, dcnt = 0;
+      for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+        const int4 it = a.items[w / a.mtiles];
+        const int N = max(16, (it.z + 15) & ~15);
+        const uint32_t idesc = umma_idesc_bf16(128, N);
+        const int db = dcnt & 1;
+        waitb(&B.dempty[db], ((dcnt >> 1) & 1) ^ 1, B, a.status);
+        tc_fence_after();
+        for (int kc = 0; kc < a.kchunks; ++kc, ++cnt, ++acnt) {
+          const int s = cnt % kStages, sa = acnt % kAStages;
+          waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
+          waitb(&B.afull[sa], (acnt / kAStages) & 1, B, a.status);
+          tc_fence_after();
+          const uint32_t bst = smem_u32(smem + s * kStageBytes + kABytes + (1024 - kABytes % 1024) % 1024);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint64_t bdesc = umma_sdesc_sw128(bst + (j >> 2) * kBSub + (j & 3) * 32);
+            umma_ts(tbase + db * 128, tbase + kTmemA0 + sa * 64 + 8 * j, bdesc, idesc, (kc | j) != 0);
+          }
+          umma_commit(&B.aempty[sa]);
+          umma_commit(&B.empty[s]);
+        }
+        umma_commit(&B.dfull[db]);
+        ++dcnt;
+      }
+      // all MMAs issued by this thread have completed before tensor memory is released
+      umma_commit(&B.done);
+      if (!mbar_wait(&B.done, 0)) set_status(a.status, kStatusTimeout);
+    }
+  } else if (warp < kWarpEpi0) {
+    // ---- dequant warps: 2 per TMEM lane quadrant, one 16-row unit each ----
+    const int q = warp & 3, uq = (warp - kWarpDequant0) >> 2;
+    const int unit = 2 * q + uq;
+    const uint32_t lane_base = (uint32_t)(32 * q + 16 * uq) << 16;
+    const int g = lane >> 2;
+    int cnt = 0, acnt = 0;
+    for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+      for (int kc = 0; kc < a.kchunks; ++kc, ++cnt, ++acnt) {
+        const int s = cnt % kStages, sa = acnt % kAStages;
+        waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
+        waitb(&B.aempty[sa], ((acnt / kAStages) & 1) ^ 1, B, a.status);
+        tc_fence_after();
+        const uint8_t *gp = smem + s * kStageBytes + unit * kGroupBytes;
+        const uint4 cw = lds128(gp + lane * 16);
+        const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.empty[s]);  // this warp's share of the A codes is in registers
+        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+        const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+        const uint32_t acol = tbase + lane_base + kTmemA0 + sa * 64;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t p[8];
+          decode_q2_exact(cws[blk], p);
+          uint32_t sg, sg8;
+          scale_pairs(sws[blk], sg, sg8);
+          // registers P0, P2 belong to row g, P1, P3 to row g+8
+          tmem_st_16x256b(acol + 16 * blk, bf16x2_mul(p[0], sg), bf16x2_mul(p[2], sg), bf16x2_mul(p[1], sg8),
+                          bf16x2_mul(p[3], sg8));
+          tmem_st_16x256b(acol + 16 * blk + 8, bf16x2_mul(p[4], sg), bf16x2_mul(p[6], sg), bf16x2_mul(p[5], sg8),
+                          bf16x2_mul(p[7], sg8));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.afull[sa]);
+      }
+    }
+  } else {
+    // ---- epilogue warps: one TMEM lane quadrant each ----
+    const int q = warp & 3;
+    int dcnt = 0;
+    for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+      const int4 it = a.items[w / a.mtiles];
+      const int mt = w % a.mtiles;
+      const int db = dcnt & 1;
+      waitb(&B.dfull[db], (dcnt >> 1) & 1, B, a.status);
+      tc_fence_after();
+      const int ntok = it.z;
+      for (int col0 = 0; col0 < ntok; col0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + ((uint32_t)(32 * q) << 16) + db * 128 + col0, v);
+        tmem_wait_ld();
+        const int nmax = min(32, ntok - col0);
+        if (MODE == 0) {
+          const int r = 32 * q + lane, tu = r >> 4, rho = r & 15;
+          const int i = (mt * kTileUnits + tu) * 8 + (rho & 7);
+          const int I = a.G.I;
+#pragma unroll
+          for (int n = 0; n < 32; ++n) {
+            const float up = __shfl_down_sync(0xffffffffu, __uint_as_float(v[n]), 8);
+            if (rho < 8 && n < nmax)
+              a.h_out[(size_t)(it.y + col0 + n) * I + i] = float_to_bf16_bits(silu_f(__uint_as_float(v[n])) * up);
+          }
+        } else {
+          const int H = a.G.H;
+          const int row = mt * 128 + 32 * q + lane;
+#pragma unroll
+          for (int n = 0; n < 32; ++n)
+            if (n < nmax) a.y_out[(size_t)(it.y + col0 + n) * H + row] = __uint_as_float(v[n]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.dempty[db]);
+      ++dcnt;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpProducer) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// Token rows in slot order: xs[p] = x[sorted_tok[p]] (one warp per position).
+__global__ void gather_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sorted_tok, int P, int H,
+                                   uint16_t *__restrict__ xs) {
+  const long long wg = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wg >= P) return;
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)sorted_tok[wg] * H);
+  uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)wg * H);
+  for (int i = lane; i < H / 8; i += 32) dst[i] = src[i];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major bf16 matrix [rows][cols], boxes of 16 rows x 64 columns, 128-byte swizzle.
+bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t tc_smem_bytes() { return (size_t)kStages * kStageBytes + sizeof(Bars) + 1024; }
+
+cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
+                              const uint16_t *x, int T, const Workspace &ws, cudaStream_t s) {
+  const int P = T * d.top_k + T;  // sorted positions (routed + shared)
+  trace_mark(MOE_KERNEL_GATHER, false, s);
+  gather_rows_kernel<<<(unsigned)(((long long)P * 32 + 255) / 256), 256, 0, s>>>(x, ws.sorted_tok, P, G.H, ws.xs);
+  trace_mark(MOE_KERNEL_GATHER, true, s);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+
+  int dev = 0, n_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const size_t smem = tc_smem_bytes();
+  TcArgs a{};
+  a.experts = experts;
+  a.shared = shared;
+  a.G = G;
+  a.E = d.n_experts;
+  a.items = ws.tc_items;
+  a.n_items = ws.n_tc_items;
+  a.status = ws.status;
+  a.h_out = ws.h;
+  a.y_out = ws.y;
+
+  CUtensorMap map_x, map_h;
+  if (!make_rows_map(&map_x, ws.xs, P, G.H) || !make_rows_map(&map_h, ws.h, P, G.I)) return cudaErrorInvalidValue;
+
+  // gate/up + SwiGLU: M = 2I interleaved rows (8 gate + 8 up per unit), K = H
+  a.mtiles = G.gu_units / kTileUnits;
+  a.kchunks = G.gu_groups;
+  a.unit_bytes = G.gu_unit_bytes;
+  a.sec_off = 0;
+  err = cudaFuncSetAttribute(tc_expert_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  trace_mark(MOE_KERNEL_GATE_UP, false, s);
+  tc_expert_kernel<0><<<n_sm, kThreadsTC, smem, s>>>(map_x, a);
+  trace_mark(MOE_KERNEL_GATE_UP, true, s);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+
+  // down: M = H rows, K = I
+  a.mtiles = G.dn_units / kTileUnits;
+  a.kchunks = G.dn_groups;
+  a.unit_bytes = G.dn_unit_bytes;
+  a.sec_off = G.gu_bytes;
+  err = cudaFuncSetAttribute(tc_expert_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  trace_mark(MOE_KERNEL_DOWN, false, s);
+  tc_expert_kernel<1><<<n_sm, kThreadsTC, smem, s>>>(map_h, a);
+  trace_mark(MOE_KERNEL_DOWN, true, s);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

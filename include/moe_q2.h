@@ -171,7 +171,8 @@ enum {
   MOE_KERNEL_GATE_UP = 5,
   MOE_KERNEL_DOWN = 6,
   MOE_KERNEL_COMBINE = 7,
-  MOE_KERNEL_DECODE_FUSED = 8
+  MOE_KERNEL_DECODE_FUSED = 8,
+  MOE_KERNEL_GATHER = 9
 };
 moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after);
 
