@@ -50,7 +50,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_sw = take(slots * 4);
   const int max_items = max_items_for(d, T, 8);
   const size_t o_items = take((size_t)max_items * 16);
-  const int max_tc_items = max_items_for(d, T, 128);
+  const int max_tc_items = max_items_for(d, T, 64);
   const size_t o_tc_items = take((size_t)max_tc_items * 16);
   const size_t o_xs = take(T > 8 ? slots * H * 2 : 0);
   const size_t o_h = take(slots * I * 2);

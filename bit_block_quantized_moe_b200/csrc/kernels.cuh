@@ -23,7 +23,7 @@ struct Workspace {
   int32_t *sorted_tok;     // [T*k + T]: token of each sorted position (shared slots last)
   float *sorted_w;         // [T*k + T]
   int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)
-  int4 *tc_items;          // [max_tc_items]: (expert, first position, tokens <= 128, 0)
+  int4 *tc_items;          // [max_tc_items]: (expert, first position, tokens <= 64, 0)
   uint32_t *n_tc_items;
   uint16_t *xs;            // [T*k + T][H] bf16 token rows in sorted-position order
   uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position

@@ -2,13 +2,15 @@
 // (tcgen05, sm_100a).
 //
 // One persistent CTA per SM walks a list of work items (expert, 128-row M
-// tile, up to 128 tokens).  For each 128-wide K chunk:
-//   producer warp   : bulk-copies the tile's packed Q2 codes + scales (8 units
-//                     x 640 B) and TMA-loads the chunk of the expert's token
-//                     rows (slot-sorted activations, 128-byte swizzle) into a
-//                     shared-memory stage;
-//   8 dequant warps : decode the codes in registers to bf16 d * (q - 1) and
-//                     store them into a tensor-memory A stage (tcgen05.st);
+// tile, up to 64 tokens).  For each 128-wide K chunk:
+//   producer warp    : one TMA load of the tile's packed Q2 codes + scales (8
+//                      units x 640 B, a 4-D tensor map over the experts) and
+//                      two of the expert's token rows (slot-sorted
+//                      activations, 128-byte swizzle, 16/32/64-row boxes)
+//                      into a shared-memory stage;
+//   16 dequant warps : decode the codes in registers to bf16 d * (q - 1) and
+//                      store them into a tensor-memory A stage (tcgen05.st),
+//                      two blocks of one 16-row unit per warp;
 //   MMA warp        : 8 x tcgen05.mma (A from tensor memory, B from shared
 //                     memory), fp32 accumulators in tensor memory, commits
 //                     release the stages;
@@ -26,24 +28,25 @@ namespace moe {
 
 namespace {
 
-constexpr int kStages = 4;         // shared-memory stages (A codes + B rows)
-constexpr int kAStages = 4;        // tensor-memory A stages
+constexpr int kStages = 8;         // shared-memory stages (A codes + B rows)
+constexpr int kAStages = 6;        // tensor-memory A stages
 constexpr int kTileUnits = 8;      // 16-row units per 128-row M tile
+constexpr int kMaxN = 64;          // tokens per work item
 constexpr int kABytes = kTileUnits * kGroupBytes;  // 5120
-constexpr int kBBox = 2048;        // one TMA box: 16 rows x 128 bytes
-constexpr int kBSub = 8 * kBBox;   // one 64-wide K half of the chunk, 128 rows: 16 KB
-constexpr int kStageBytes = 1024 * ((kABytes + 2 * kBSub + 1023) / 1024);  // 37888
-constexpr int kWarpProducer = 0, kWarpMMA = 1, kWarpDequant0 = 2, kNumDequant = 8, kWarpEpi0 = 10, kNumEpi = 4;
-constexpr int kThreadsTC = (kWarpEpi0 + kNumEpi) * 32;  // 448
+constexpr int kBSub = kMaxN * 128;                 // one 64-wide K half of the chunk: 8 KB
+constexpr int kStageBytes = kABytes + 2 * kBSub;   // 21504 (a multiple of 1024)
+constexpr int kWarpProducer = 0, kWarpMMA = 1, kWarpDequant0 = 2, kNumDequant = 16, kWarpEpi0 = 18, kNumEpi = 4;
+constexpr int kThreadsTC = (kWarpEpi0 + kNumEpi) * 32;  // 704
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemA0 = 256;  // A stages live at columns 256 + 64 * sa; D buffers at 0 and 128
+constexpr uint32_t kTmemA0 = 128;  // D buffers at columns 0 and 64; A stages at 128 + 64 * sa
+static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment for the 128-byte swizzle");
 
 struct TcArgs {
   const uint8_t *experts;
   const uint8_t *shared;
   PackedGeom G;
   int E;
-  const int4 *items;          // (expert or E for shared, first sorted position, tokens <= 128, 0)
+  const int4 *items;          // (expert or E for shared, first sorted position, tokens <= 64, 0)
   const uint32_t *n_items;
   int mtiles;                 // 128-row tiles per expert for this projection
   int kchunks;                // 128-wide K chunks (block groups)
@@ -83,8 +86,14 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   return d;
 }
 
+struct TcMaps {
+  CUtensorMap a_routed;  // packed units of the routed experts, 4-D (u32 in unit group, group, unit, expert)
+  CUtensorMap a_shared;  // the shared expert, same shape with one expert
+  CUtensorMap b[3];      // token rows [positions][K] bf16, boxes of 16 / 32 / 64 rows x 64 columns
+};
+
 template <int MODE>  // 0: gate/up + SwiGLU -> h (bf16); 1: down -> y (fp32)
-__global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+__global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_constant__ TcMaps maps, TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   Bars &B = *reinterpret_cast<Bars *>(smem + kStages * kStageBytes);
@@ -121,21 +130,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
         const int4 it = a.items[w / a.mtiles];
         const int mt = w % a.mtiles;
-        const int nb = (it.z + 15) >> 4;  // 16-row boxes
-        const uint8_t *ex = it.x == a.E ? a.shared : a.experts + (size_t)it.x * a.G.expert_bytes;
-        const uint8_t *abase = ex + a.sec_off + (size_t)mt * kTileUnits * a.unit_bytes;
+        const int bsel = it.z <= 16 ? 0 : (it.z <= 32 ? 1 : 2);
+        const int nrows = 16 << bsel;
+        const CUtensorMap *amap = it.x == a.E ? &maps.a_shared : &maps.a_routed;
+        const int ae = it.x == a.E ? 0 : it.x;
         for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
           const int s = cnt % kStages;
           if (!waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) continue;
           uint8_t *st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&B.full[s], (uint32_t)(kABytes + nb * 2 * kBBox));
-          for (int u = 0; u < kTileUnits; ++u)
-            bulk_g2s(st + u * kGroupBytes, abase + (size_t)u * a.unit_bytes + (size_t)kc * kGroupBytes, kGroupBytes,
-                     &B.full[s]);
-          uint8_t *bst = st + kABytes + (1024 - kABytes % 1024) % 1024;
+          mbar_arrive_expect_tx(&B.full[s], (uint32_t)(kABytes + 2 * nrows * 128));
+          tma_load_4d(st, amap, 0, kc, mt * kTileUnits, ae, &B.full[s]);
           for (int sub = 0; sub < 2; ++sub)
-            for (int b = 0; b < nb; ++b)
-              tma_load_2d(bst + sub * kBSub + b * kBBox, &tmB, kc * 128 + sub * 64, it.y + 16 * b, &B.full[s]);
+            tma_load_2d(st + kABytes + sub * kBSub, &maps.b[bsel], kc * 128 + sub * 64, it.y, &B.full[s]);
         }
       }
       // every copy issued must land before the CTA exits
@@ -156,11 +162,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
           waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
           waitb(&B.afull[sa], (acnt / kAStages) & 1, B, a.status);
           tc_fence_after();
-          const uint32_t bst = smem_u32(smem + s * kStageBytes + kABytes + (1024 - kABytes % 1024) % 1024);
+          const uint32_t bst = smem_u32(smem + s * kStageBytes + kABytes);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint64_t bdesc = umma_sdesc_sw128(bst + (j >> 2) * kBSub + (j & 3) * 32);
-            umma_ts(tbase + db * 128, tbase + kTmemA0 + sa * 64 + 8 * j, bdesc, idesc, (kc | j) != 0);
+            umma_ts(tbase + db * kMaxN, tbase + kTmemA0 + sa * 64 + 8 * j, bdesc, idesc, (kc | j) != 0);
           }
           umma_commit(&B.aempty[sa]);
           umma_commit(&B.empty[s]);
@@ -173,8 +179,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       if (!mbar_wait(&B.done, 0)) set_status(a.status, kStatusTimeout);
     }
   } else if (warp < kWarpEpi0) {
-    // ---- dequant warps: 2 per TMEM lane quadrant, one 16-row unit each ----
-    const int q = warp & 3, uq = (warp - kWarpDequant0) >> 2;
+    // ---- dequant warps: 4 per TMEM lane quadrant = 2 units x 2 block pairs ----
+    const int dw = warp - kWarpDequant0;
+    const int q = warp & 3, uq = (dw >> 2) & 1, bh = dw >> 3;
     const int unit = 2 * q + uq;
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * uq) << 16;
     const int g = lane >> 2;
@@ -186,23 +193,23 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         waitb(&B.aempty[sa], ((acnt / kAStages) & 1) ^ 1, B, a.status);
         tc_fence_after();
         const uint8_t *gp = smem + s * kStageBytes + unit * kGroupBytes;
-        const uint4 cw = lds128(gp + lane * 16);
-        const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
+        const uint2 cw = *reinterpret_cast<const uint2 *>(gp + lane * 16 + 8 * bh);
+        const uint2 sw = *reinterpret_cast<const uint2 *>(gp + kGroupCodeBytes + g * 16 + 8 * bh);
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.empty[s]);  // this warp's share of the A codes is in registers
-        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
-        const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
-        const uint32_t acol = tbase + lane_base + kTmemA0 + sa * 64;
+        const uint32_t cws[2] = {cw.x, cw.y};
+        const uint32_t sws[2] = {sw.x, sw.y};
+        const uint32_t acol = tbase + lane_base + kTmemA0 + sa * 64 + 32 * bh;
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int bb = 0; bb < 2; ++bb) {
           uint32_t p[8];
-          decode_q2_exact(cws[blk], p);
+          decode_q2_exact(cws[bb], p);
           uint32_t sg, sg8;
-          scale_pairs(sws[blk], sg, sg8);
+          scale_pairs(sws[bb], sg, sg8);
           // registers P0, P2 belong to row g, P1, P3 to row g+8
-          tmem_st_16x256b(acol + 16 * blk, bf16x2_mul(p[0], sg), bf16x2_mul(p[2], sg), bf16x2_mul(p[1], sg8),
+          tmem_st_16x256b(acol + 16 * bb, bf16x2_mul(p[0], sg), bf16x2_mul(p[2], sg), bf16x2_mul(p[1], sg8),
                           bf16x2_mul(p[3], sg8));
-          tmem_st_16x256b(acol + 16 * blk + 8, bf16x2_mul(p[4], sg), bf16x2_mul(p[6], sg), bf16x2_mul(p[5], sg8),
+          tmem_st_16x256b(acol + 16 * bb + 8, bf16x2_mul(p[4], sg), bf16x2_mul(p[6], sg), bf16x2_mul(p[5], sg8),
                           bf16x2_mul(p[7], sg8));
         }
         tmem_wait_st();
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       const int ntok = it.z;
       for (int col0 = 0; col0 < ntok; col0 += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + ((uint32_t)(32 * q) << 16) + db * 128 + col0, v);
+        tmem_ld_32x32b_x32(tbase + ((uint32_t)(32 * q) << 16) + db * kMaxN + col0, v);
         tmem_wait_ld();
         const int nmax = min(32, ntok - col0);
         if (MODE == 0) {
@@ -282,17 +289,45 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major bf16 matrix [rows][cols], boxes of 16 rows x 64 columns, 128-byte swizzle.
-bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols) {
+// 2-D map over a row-major bf16 matrix [rows][cols], boxes of box_rows x 64 columns, 128-byte swizzle.
+bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D map over packed units: (32-bit word within a 640-byte block group, group, unit, expert);
+// one box is one group of 8 consecutive units (5120 bytes, no swizzle).
+bool make_units_map(CUtensorMap *map, const void *base, int groups, int units, int experts, size_t unit_bytes,
+                    size_t expert_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {kGroupBytes / 4, (cuuint64_t)groups, (cuuint64_t)units, (cuuint64_t)experts};
+  const cuuint64_t strides[3] = {kGroupBytes, unit_bytes, expert_bytes};
+  const cuuint32_t box[4] = {kGroupBytes / 4, 1, kTileUnits, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_maps(TcMaps *m, const uint8_t *experts, const uint8_t *shared, const PackedGeom &G, int E, bool down,
+               const void *rows, int P) {
+  const int groups = down ? G.dn_groups : G.gu_groups;
+  const int units = down ? G.dn_units : G.gu_units;
+  const size_t ub = down ? G.dn_unit_bytes : G.gu_unit_bytes;
+  const size_t off = down ? G.gu_bytes : 0;
+  const int K = down ? G.I : G.H;
+  bool ok = make_units_map(&m->a_routed, experts + off, groups, units, E, ub, G.expert_bytes) &&
+            make_units_map(&m->a_shared, shared + off, groups, units, 1, ub, G.expert_bytes);
+  for (int i = 0; i < 3 && ok; ++i) ok = make_rows_map(&m->b[i], rows, P, K, 16 << i);
+  return ok;
 }
 
 }  // namespace
@@ -323,8 +358,10 @@ cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint
   a.h_out = ws.h;
   a.y_out = ws.y;
 
-  CUtensorMap map_x, map_h;
-  if (!make_rows_map(&map_x, ws.xs, P, G.H) || !make_rows_map(&map_h, ws.h, P, G.I)) return cudaErrorInvalidValue;
+  TcMaps maps_gu, maps_dn;
+  if (!make_maps(&maps_gu, experts, shared, G, d.n_experts, false, ws.xs, P) ||
+      !make_maps(&maps_dn, experts, shared, G, d.n_experts, true, ws.h, P))
+    return cudaErrorInvalidValue;
 
   // gate/up + SwiGLU: M = 2I interleaved rows (8 gate + 8 up per unit), K = H
   a.mtiles = G.gu_units / kTileUnits;
@@ -334,7 +371,7 @@ cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint
   err = cudaFuncSetAttribute(tc_expert_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   trace_mark(MOE_KERNEL_GATE_UP, false, s);
-  tc_expert_kernel<0><<<n_sm, kThreadsTC, smem, s>>>(map_x, a);
+  tc_expert_kernel<0><<<n_sm, kThreadsTC, smem, s>>>(maps_gu, a);
   trace_mark(MOE_KERNEL_GATE_UP, true, s);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -347,7 +384,7 @@ cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint
   err = cudaFuncSetAttribute(tc_expert_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   trace_mark(MOE_KERNEL_DOWN, false, s);
-  tc_expert_kernel<1><<<n_sm, kThreadsTC, smem, s>>>(map_h, a);
+  tc_expert_kernel<1><<<n_sm, kThreadsTC, smem, s>>>(maps_dn, a);
   trace_mark(MOE_KERNEL_DOWN, true, s);
   return cudaGetLastError();
 }

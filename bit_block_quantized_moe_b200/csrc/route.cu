@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
   if (!is_last) return;
   __threadfence();
   // Work items: (expert, first sorted position, tokens) in tiles of 8 tokens
-  // (register-dequant path) and of 128 tokens (tcgen05 path).
+  // (register-dequant path) and of 64 tokens (tcgen05 path).
   __shared__ int s_cnt[256], s_items[256], s_tc[256];
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int eb = threadIdx.x * per, ee = min(E, eb + per);
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
     const int c = ((volatile int32_t *)counts)[i];
     my_cnt += c;
     my_items += (c + 7) >> 3;
-    my_tc += (c + 127) >> 7;
+    my_tc += (c + 63) >> 6;
   }
   s_cnt[threadIdx.x] = my_cnt;
   s_items[threadIdx.x] = my_items;
@@ -307,8 +307,8 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
     const int shared_items = (T + 7) >> 3;
     for (int i = 0; i < shared_items; ++i) items[b + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
     *n_items = (uint32_t)(b + shared_items);
-    const int shared_tc = (T + 127) >> 7;
-    for (int i = 0; i < shared_tc; ++i) tc_items[tc + i] = make_int4(E, T * k + 128 * i, min(128, T - 128 * i), 0);
+    const int shared_tc = (T + 63) >> 6;
+    for (int i = 0; i < shared_tc; ++i) tc_items[tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
     *n_tc_items = (uint32_t)(tc + shared_tc);
   }
   __syncthreads();
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
     const int c = ((volatile int32_t *)counts)[i];
     offsets[i] = pos;
     for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
-    for (int j = 0; j < c; j += 128) tc_items[itc++] = make_int4(i, pos + j, min(128, c - j), 0);
+    for (int j = 0; j < c; j += 64) tc_items[itc++] = make_int4(i, pos + j, min(64, c - j), 0);
     pos += c;
   }
 }
