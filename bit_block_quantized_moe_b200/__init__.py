@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     moe_packed_expert_bytes,
     moe_rmsnorm_residual,
     moe_route,
+    moe_route_noalloc,
     moe_status_str,
     moe_trace_kernel,
     MOE_KERNEL,

@@ -42,6 +42,7 @@ EXPORTED = [
     "moe_pack_q2",
     "moe_workspace_bytes",
     "moe_route",
+    "moe_route_noalloc",
     "moe_layer_forward",
     "moe_experts_forward",
     "moe_rmsnorm_residual",
@@ -70,6 +71,8 @@ def lib():
         L.moe_workspace_bytes.argtypes = [D, i32]
         L.moe_route.restype = ctypes.c_int
         L.moe_route.argtypes = [D, P, ctypes.POINTER(moe_router), i32, P, P, P, sz, P]
+        L.moe_route_noalloc.restype = ctypes.c_int
+        L.moe_route_noalloc.argtypes = [D, P, ctypes.POINTER(moe_router), i32, P, P, P]
         L.moe_layer_forward.restype = ctypes.c_int
         L.moe_layer_forward.argtypes = [D, P, ctypes.POINTER(moe_router), ctypes.POINTER(moe_experts),
                                         ctypes.POINTER(moe_shared), P, i32, P, P, P, sz, P]
@@ -143,6 +146,15 @@ def moe_route(dims, x, router_w, router_b, T: int, topk_idx, topk_w, workspace, 
                            _ptr(topk_w), _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream(stream))
     _check(code, "moe_route")
+
+
+def moe_route_noalloc(dims, x, router_w, router_b, T: int, topk_idx, topk_w, stream=None):
+    """moe_route without a workspace: the library's own static device scratch holds the
+    logits, for callers that cannot allocate device memory (see include/moe_q2.h)."""
+    r = moe_router(_ptr(router_w), _ptr(router_b))
+    code = lib().moe_route_noalloc(ctypes.byref(_dims(dims)), _ptr(x), ctypes.byref(r), int(T), _ptr(topk_idx),
+                                   _ptr(topk_w), _stream(stream))
+    _check(code, "moe_route_noalloc")
 
 
 def moe_layer_forward(dims, x, router_w, router_b, experts_packed, shared_packed, out, T: int, workspace,

@@ -122,6 +122,30 @@ size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T);
 moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_router *router, int32_t T,
                      int32_t *topk_idx, float *topk_w, void *workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- routing without a workspace --------------------------------------------------
+ * The paper has no counterpart to this entry point; it exists for callers of
+ * this library that cannot allocate device memory: code running inside a
+ * stream capture, where a cudaMalloc would break the capture; engines whose
+ * device memory is reserved up front by their own pool, with nothing left to
+ * hand out; and latency-bound loops that cannot afford an allocation's
+ * implicit device synchronisation.
+ * It computes exactly what moe_route computes (same kernels, same results),
+ * but the scratch those kernels need -- the [T, n_experts] fp32 router logits
+ * -- lives in a file-scope device array of MOE_NOALLOC_MAX_LOGITS floats
+ * (1 MiB) inside this library, which every GPU that loads the library holds
+ * until the process exits.  The call allocates nothing.
+ *  - T * n_experts > MOE_NOALLOC_MAX_LOGITS returns MOE_ERR_WORKSPACE.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array: calls that overlap on the GPU (different
+ *    streams, or different host threads) race and may return each other's
+ *    routing.  Nothing in the array needs to start at zero: every call
+ *    rewrites the logits it reads.
+ * Arguments as moe_route, minus the workspace. */
+#define MOE_NOALLOC_MAX_LOGITS 262144
+moe_status moe_route_noalloc(const moe_dims *dims, const uint16_t *x, const moe_router *router, int32_t T,
+                             int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
 /* ---- the layer ------------------------------------------------------------------
  * out[t] = shared(x[t]) + sum_j w[t,j] * expert_{idx[t,j]}(x[t]), with
  * expert(v) = Wd (silu(Wg v) * (Wu v)) and silu(z) = z / (1 + exp(-z)).
