@@ -95,7 +95,8 @@ struct TcMaps {
 template <int MODE>  // 0: gate/up + SwiGLU -> h (bf16); 1: down -> y (fp32)
 __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_constant__ TcMaps maps, TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned start (pointer arithmetic on the shared array keeps shared-memory addressing)
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars &B = *reinterpret_cast<Bars *>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = (int)*a.n_items;
