@@ -140,51 +140,96 @@ __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t
   if (threadIdx.x < T) logits[(size_t)threadIdx.x * E + e] = router_combine(part[threadIdx.x], bias ? bias[e] : 0.f);
 }
 
-// Many tokens: 64 tokens x 64 experts per CTA, fp32 FMA tiles through shared memory.
-__global__ void __launch_bounds__(256) router_logits_tiled_kernel(const uint16_t *__restrict__ x,
-                                                                   const float *__restrict__ Wr,
-                                                                   const float *__restrict__ bias, int T, int H,
-                                                                   int E, float *__restrict__ logits,
-                                                                   uint32_t *zero_p, size_t zero_n) {
+// Many tokens: tensor cores with an exact 3-way bf16 split of the fp32 router
+// weights.  w = hi + mid + lo exactly (each a bf16 holding the next 8
+// significant bits); x is bf16 already, so every product is exact in fp32 and
+// only the fp32 accumulation rounds, as in a CUDA-core dot product.  Each
+// 256-wide K slice is accumulated in a fresh tensor-core accumulator and then
+// added to the running fp32 sum.  CTA tile: 64 experts x 64 tokens, 8 warps of
+// 16 experts x 32 tokens (m16n8k16).
+__device__ __forceinline__ void split3_bf16(float w, uint16_t &hi, uint16_t &mid, uint16_t &lo) {
+  hi = float_to_bf16_bits(w);
+  const float r1 = w - bf16_bits_to_float(hi);
+  mid = float_to_bf16_bits(r1);
+  const float r2 = r1 - bf16_bits_to_float(mid);
+  lo = float_to_bf16_bits(r2);
+}
+
+__global__ void __launch_bounds__(256) router_logits_mma_kernel(const uint16_t *__restrict__ x,
+                                                                 const float *__restrict__ Wr,
+                                                                 const float *__restrict__ bias, int T, int H, int E,
+                                                                 float *__restrict__ logits, uint32_t *zero_p,
+                                                                 size_t zero_n) {
   clear_range(zero_p, zero_n);
-  __shared__ float xs[32][68];
-  __shared__ float ws[32][68];
-  const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  constexpr int BK = 32, WS = BK + 4, XS = BK + 8;  // padded row strides (floats / halves)
+  __shared__ float ws[64 * WS];
+  __shared__ uint16_t xs[64 * XS];
+  const int e0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const int wm = warp & 3, wn = warp >> 2;
   float acc[4][4] = {};
-  for (int k0 = 0; k0 < H; k0 += 32) {
-    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
-      const int row = i >> 5, kk = i & 31;
-      const int t = t0 + row, e = e0 + row;
-      xs[kk][row] = t < T ? bf16_bits_to_float(x[(size_t)t * H + k0 + kk]) : 0.f;
-      ws[kk][row] = e < E ? Wr[(size_t)e * H + k0 + kk] : 0.f;
+  float part[4][4] = {};
+  for (int k0 = 0; k0 < H; k0 += BK) {
+    // stage 64 x 32 router weights and 64 x 32 tokens
+    for (int i = threadIdx.x; i < 64 * (BK / 4); i += 256) {
+      const int r = i / (BK / 4), c4 = i % (BK / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0 + r < E) v = *reinterpret_cast<const float4 *>(Wr + (size_t)(e0 + r) * H + k0 + 4 * c4);
+      *reinterpret_cast<float4 *>(ws + r * WS + 4 * c4) = v;
+    }
+    for (int i = threadIdx.x; i < 64 * (BK / 8); i += 256) {
+      const int r = i / (BK / 8), c8 = i % (BK / 8);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (t0 + r < T) v = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + r) * H + k0 + 8 * c8);
+      *reinterpret_cast<uint2 *>(xs + r * XS + 8 * c8) = make_uint2(v.x, v.y);
+      *reinterpret_cast<uint2 *>(xs + r * XS + 8 * c8 + 4) = make_uint2(v.z, v.w);
     }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 32; ++kk) {
-      float a[4], b[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = xs[kk][ty * 4 + i];
-        b[i] = ws[kk][tx * 4 + i];
+    for (int kk = 0; kk < BK; kk += 16) {
+      // A fragments of the three splits: rows wm*16 + g (+8), k = kk + 2c (+1) and kk + 2c + 8 (+9)
+      uint32_t ah[4], am[4], al[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = wm * 16 + g + 8 * (q & 1), col = kk + 2 * c + 8 * (q >> 1);
+        const float2 w2 = *reinterpret_cast<const float2 *>(ws + row * WS + col);
+        uint16_t h0, m0, l0, h1, m1, l1;
+        split3_bf16(w2.x, h0, m0, l0);
+        split3_bf16(w2.y, h1, m1, l1);
+        ah[q] = h0 | ((uint32_t)h1 << 16);
+        am[q] = m0 | ((uint32_t)m1 << 16);
+        al[q] = l0 | ((uint32_t)l1 << 16);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      for (int nt = 0; nt < 4; ++nt) {
+        const uint16_t *xr = xs + (wn * 32 + nt * 8 + g) * XS + kk + 2 * c;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t *>(xr);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t *>(xr + 8);
+        mma_bf16_16816(part[nt], ah, b0, b1, part[nt]);
+        mma_bf16_16816(part[nt], am, b0, b1, part[nt]);
+        mma_bf16_16816(part[nt], al, b0, b1, part[nt]);
+      }
     }
     __syncthreads();
-  }
+    if (((k0 + BK) & 255) == 0 || k0 + BK >= H) {  // end of a 256-wide K slice
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) continue;
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
+        for (int q = 0; q < 4; ++q) {
+          acc[nt][q] += part[nt][q];
+          part[nt][q] = 0.f;
+        }
     }
   }
+  // D fragment: (row g, cols 2c, 2c+1), (row g+8, cols 2c, 2c+1); rows = experts, cols = tokens
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = e0 + wm * 16 + g + 8 * (q >> 1);
+      const int t = t0 + wn * 32 + nt * 8 + 2 * c + (q & 1);
+      if (e < E && t < T) logits[(size_t)t * E + e] = acc[nt][q] + (bias ? bias[e] : 0.f);
+    }
 }
 
 // Top-k per token, one warp per token (see warp_topk); optionally marks the
@@ -222,8 +267,7 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, 
   } else {
     dim3 grid((E + 63) / 64, (T + 63) / 64);
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
-    router_logits_tiled_kernel<<<grid, 256, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin,
-                                                     ws.zero_words);
+    router_logits_mma_kernel<<<grid, 256, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin, ws.zero_words);
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
   }
   cudaError_t err = cudaGetLastError();
