@@ -14,7 +14,7 @@
 //     gate/up units (expert, 8 intermediate rows) and down pairs (expert, 16
 //     output rows).  The producer streams the CTA's units into a ring of
 //     shared-memory stages as stages free up; stage s belongs to consumer
-//     warp s % 14, which computes the whole unit (full K) with no cross-warp
+//     warp s % min(14, stages), which computes the whole unit (full K) with no cross-warp
 //     reduction and writes h = silu(g) * u (bf16) straight from its
 //     accumulators.  At the end the CTA publishes, per expert, how many of
 //     its units are done.
@@ -24,10 +24,14 @@
 //     partial = w[t, e] * (Wd_e h_e) per (expert, tile).  The last CTA to
 //     contribute to a tile sums its partials in expert order and writes out
 //     (bf16).
-// Dequantisation happens in registers and feeds m16n8k16 tensor-core MMAs
-// with the tokens as the 8 columns; gate/up uses the biased decode with the
-// -1 offset folded into the accumulator start (decode_q2_biased), down the
-// exact decode.  Every wait is bounded (sync.cuh).
+// Weights reach the tensor cores with no arithmetic: the 2-bit codes of a
+// row are masked into e4m3 bytes (value q * 2^-9) that form the A fragment of
+// an m16n8k32 fp8 MMA.  The tokens form the B fragment: each token vector is
+// scaled by a power of two and split into two e4m3 terms (columns 2t and
+// 2t+1, 4 tokens per MMA), exact for every element above 2^-8 of the
+// vector's largest.  The -1 of d * (q - 1) starts the accumulator at minus the
+// block sum of the token, and the fp16 block scale d multiplies each block's
+// fp32 result.  Every wait is bounded (sync.cuh).
 #include "kernels.cuh"
 #include "router.cuh"
 #include "sync.cuh"
@@ -68,8 +72,12 @@ struct DecodeArgs {
 };
 
 struct SmemLayout {
-  uint32_t bars, xs, corr, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc, ring, total;
+  uint32_t bars, xs, corr, xb, xsc, hb, hcorr, hsc, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc,
+      ring, total;
 };
+
+// Token quads: the 8 columns of an m16n8k32 MMA hold 4 tokens x 2 split terms.
+__host__ __device__ inline int token_quads(int T) { return (T + 3) / 4; }
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
@@ -78,14 +86,25 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   uint32_t o = 0;
   L.bars = o;  // full[ns], empty[ns], rbar, xbar
   o = align_to(o + 8u * (2 * ns + 2), 16);
+  // xs: the tokens (bf16 rows, phase A).  The same bytes hold the h fragments of phase D.
+  const uint32_t hb_bytes = 2u * token_quads(T) * (kMaxI / 32) * 256;
+  const uint32_t hcorr_bytes = 2u * (kMaxI / 32) * kMaxTok * 4;
+  const uint32_t xs_bytes = (uint32_t)T * (H + 16) * 2;
   L.xs = o;
-  o = align_to(o + (uint32_t)T * (H + 16) * 2, 16);
-  L.corr = o;
+  L.hb = o;  // [2 cached experts][quads][I/32][32] B fragments of h
+  L.hcorr = o + hb_bytes;  // [2][I/32][8]
+  L.hsc = L.hcorr + hcorr_bytes;  // [2][8]
+  o = align_to(o + max(xs_bytes, hb_bytes + hcorr_bytes + 2u * kMaxTok * 4), 16);
+  L.corr = o;  // [H/32 blocks][8 tokens]: -2^-9 * sum of the scaled tokens over the block
   o = align_to(o + (uint32_t)(H / 32) * kMaxTok * 4, 16);
+  L.xb = o;  // [quads][H/32 blocks][32 lanes] B fragments (uint2) of the scaled, split tokens
+  o = align_to(o + (uint32_t)token_quads(T) * (H / 32) * 256, 16);
+  L.xsc = o;  // [8] 2^(9 - s_t): undoes the token scale and the 2^-9 of the A bytes
+  o += kMaxTok * 4;
   L.rpart = o;  // [rows per pass <= 4][8 tokens][4 quarters]
   o += 4 * kMaxTok * 4 * 4;
-  L.red = o;    // top-k scratch (phase B), then the h cache of phase D: [2 entries][8 tokens][I + 16]
-  o += align_to(2u * kMaxTok * (kMaxI + 16) * 2, 16);
+  L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
+  o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
   L.sel_idx = o;
   o += kMaxSel * 4;
   L.sel_w = o;
@@ -100,15 +119,135 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   o = align_to(o + kMaxEntries * kMaxTok, 16);
   L.tokw = o;
   o = align_to(o + kMaxEntries * kMaxTok * 4, 16);
-  L.misc = o;
-  o += 32;
+  L.misc = o;  // [0] entries [1] abort [2] barrier flag [3] done tiles [8..15] token scale exponents
+  o += 64;
   L.ring = align_to(o, 128);
   L.total = L.ring + (uint32_t)ns * stage_bytes;
   return L;
 }
 
-// B-operand scale 1/4 for the fragment registers of k pair (4c+2, 4c+3); exact.
-__device__ __forceinline__ uint32_t bf16x2_quarter(uint32_t v) { return bf16x2_fma(v, 0x3E803E80u, 0x80008000u); }
+// Per-token power-of-two scales, block correction sums and e4m3 B fragments of
+// the vectors v[t][0..K) (bf16 rows `stride` elements apart), t < T.  All
+// consumer threads call it (it holds named barriers).
+//   unscale[t] = 2^(9 - s_t), with max_k |v[t][k]| * 2^s_t in [128, 256);
+//   corr[b][t] = -2^-9 * sum_{k in block b} v[t][k] * 2^s_t  (the -1 of q - 1);
+//   frag[(quad * nb + b) * 32 + lane]: lane (g, c) holds column g = 2 * (t % 4)
+//   + split term, rows k in block order e4m3_k_lo (x) / e4m3_k_hi (x, times 1/4).
+__device__ void build_b_fragments(const uint16_t *v, int stride, int K, int T, int nq, uint2 *frag, float *corr,
+                                  float *unscale, int *sexp, int warp, int lane, int tid) {
+  const int nb = K / 32;
+  if (warp < T) {
+    uint32_t m = 0;  // largest |v| as a bf16 bit pattern (ordered like the magnitudes)
+    for (int i = lane; i < K / 8; i += 32) {
+      const uint4 u = *reinterpret_cast<const uint4 *>(v + warp * stride + 8 * i);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) m = max(m, max(w[h] & 0x7FFFu, (w[h] >> 16) & 0x7FFFu));
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == 0) {
+      const int sx = e4m3_scale_exp(__uint_as_float(m << 16));
+      sexp[warp] = sx;
+      unscale[warp] = 512.f * exp2_int(-sx);
+    }
+  }
+  named_bar(kBarConsumers, kConsumers);
+  for (int i = tid; i < nb * kMaxTok; i += kConsumers) {
+    const int b = i / kMaxTok, t = i % kMaxTok;
+    float sum = 0.f;
+    if (t < T) {
+      const float sc = exp2_int(sexp[t]);
+      const uint4 *row = reinterpret_cast<const uint4 *>(v + t * stride + 32 * b);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 u = row[q];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          sum = fmaf(__uint_as_float(w[h] << 16), sc, sum);
+          sum = fmaf(__uint_as_float(w[h] & 0xffff0000u), sc, sum);
+        }
+      }
+    }
+    corr[b * kMaxTok + t] = -sum * (1.f / 512.f);
+  }
+  for (int i = tid; i < nq * nb * 32; i += kConsumers) {
+    const int qd = i / (nb * 32), r = i % (nb * 32), b = r / 32, ln = r % 32;
+    const int gq = ln >> 2, cq = ln & 3, t = 4 * qd + (gq >> 1), part = gq & 1;
+    uint2 f = make_uint2(0u, 0u);
+    if (t < T) {
+      const float sc = exp2_int(sexp[t]);
+      const uint16_t *row = v + t * stride + 32 * b;
+      float lo[4], hi[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float vl = bf16_bits_to_float(row[e4m3_k_lo(cq, j)]) * sc;
+        const float vh = bf16_bits_to_float(row[e4m3_k_hi(cq, j)]) * sc * 0.25f;
+        const float hl = e4m3_split_hi(vl), hh = e4m3_split_hi(vh);
+        lo[j] = part ? vl - hl : hl;
+        hi[j] = part ? vh - hh : hh;
+      }
+      f.x = pack_e4m3x4(lo[0], lo[1], lo[2], lo[3]);
+      f.y = pack_e4m3x4(hi[0], hi[1], hi[2], hi[3]);
+    }
+    frag[i] = f;
+  }
+  named_bar(kBarConsumers, kConsumers);
+}
+
+// One 16-row unit over n_groups block groups: acc[quad][r] with r = (row g,
+// split 0), (row g, split 1), (row g+8, split 0), (row g+8, split 1) of token
+// 4 * quad + c, in units of 2^(s_t - 9).  Four block tiles per group are
+// staged: loads, code masking, one m16n8k32 MMA per quad (accumulator started
+// at the block's correction), then the fp16 block scales.
+template <int NQ>
+__device__ __forceinline__ void unit_gemv(const uint8_t *st, int n_groups, const uint2 *frag, const float *corr,
+                                          int lane, float (&acc)[2][4]) {
+  const int g = lane >> 2, c = lane & 3;
+  const int nb = n_groups * 4;
+#pragma unroll
+  for (int qd = 0; qd < 2; ++qd)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[qd][r] = 0.f;
+  for (int grp = 0; grp < n_groups; ++grp) {
+    const uint8_t *gp = st + (size_t)grp * kGroupBytes;
+    const uint4 cw = lds128(gp + lane * 16);
+    const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
+    const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+    const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+    uint2 bf[NQ][4];
+    float cn[NQ][4];
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      const int b = grp * 4 + blk;
+#pragma unroll
+      for (int qd = 0; qd < NQ; ++qd) {
+        bf[qd][blk] = frag[(qd * nb + b) * 32 + lane];
+        cn[qd][blk] = corr[b * kMaxTok + 4 * qd + c];
+      }
+    }
+    float d[NQ][4][4];
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      uint32_t am[4];
+      decode_q2_e4m3(cws[blk], am);
+#pragma unroll
+      for (int qd = 0; qd < NQ; ++qd) {
+        const float cin[4] = {cn[qd][blk], 0.f, cn[qd][blk], 0.f};
+        mma_e4m3_16832(d[qd][blk], am, bf[qd][blk].x, bf[qd][blk].y, cin);
+      }
+    }
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
+#pragma unroll
+      for (int qd = 0; qd < NQ; ++qd) {
+        fma2_bcast(acc[qd][0], acc[qd][1], s2.x, d[qd][blk][0], d[qd][blk][1]);
+        fma2_bcast(acc[qd][2], acc[qd][3], s2.y, d[qd][blk][2], d[qd][blk][3]);
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -121,6 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   uint64_t *xbar = rbar + 1;
   uint16_t *xs = reinterpret_cast<uint16_t *>(smem + L.xs);
   float *corr = reinterpret_cast<float *>(smem + L.corr);
+  uint2 *xb = reinterpret_cast<uint2 *>(smem + L.xb);
+  float *xsc = reinterpret_cast<float *>(smem + L.xsc);
+  uint2 *hb = reinterpret_cast<uint2 *>(smem + L.hb);
+  float *hcorr = reinterpret_cast<float *>(smem + L.hcorr);
+  float *hsc = reinterpret_cast<float *>(smem + L.hsc);
+  const int nq = token_quads(T);
   float *rpart = reinterpret_cast<float *>(smem + L.rpart);
   float *red = reinterpret_cast<float *>(smem + L.red);
   int *sel_idx = reinterpret_cast<int *>(smem + L.sel_idx);
@@ -130,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   int *ent = reinterpret_cast<int *>(smem + L.ent);
   int8_t *tokj = reinterpret_cast<int8_t *>(smem + L.tokj);
   float *tokw = reinterpret_cast<float *>(smem + L.tokw);
-  int *misc = reinterpret_cast<int *>(smem + L.misc);  // [0] entries [1] abort [2] barrier flag [3] done tiles
+  int *misc = reinterpret_cast<int *>(smem + L.misc);
   uint8_t *ring = smem + L.ring;
   uint32_t *ready = a.tile_cnt + G.dn_units;
 
@@ -187,24 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     if (blockIdx.x == 0)
       for (int i = tid; i < G.dn_units + kMaxEntries; i += kConsumers) a.tile_cnt[i] = 0u;
     bounded_wait(xbar, 0);
-    // correction sums of the biased decode: C[b][t] = sum_j c_j x[t][32b + j], c_j = 129 (j%4 < 2) or 33
-    for (int i = tid; i < (H / 32) * T; i += kConsumers) {
-      const int b = i / T, t = i % T;
-      const uint4 *xr = reinterpret_cast<const uint4 *>(xs + t * xstride + 32 * b);
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = xr[q];
-        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int h2 = 0; h2 < 4; ++h2) {  // elements j = 8q + 2h2 (even) and j + 1
-          const float coef = (h2 & 1) ? 33.f : 129.f;
-          s = fmaf(coef, __uint_as_float(wd[h2] << 16), s);
-          s = fmaf(coef, __uint_as_float(wd[h2] & 0xffff0000u), s);
-        }
-      }
-      corr[b * kMaxTok + t] = s;
-    }
+    // Tokens as e4m3 B fragments: per-token power-of-two scale, two split terms.
+    build_b_fragments(xs, xstride, H, T, nq, xb, corr, xsc, misc + 8, warp, lane, tid);
     bounded_wait(rbar, 0);
     constexpr int kRowsPerPass = kConsumerWarps / 4;  // 4 warps (quarters) per router row
     for (int r0 = 0; r0 < n_rrows; r0 += kRowsPerPass) {
@@ -303,6 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const int n_gu_st = g1 - g0;
   const int n_dn_st = (d1 - d0 + pps - 1) / pps;
   const int n_st = n_gu_st + n_dn_st;
+  // Stage s is consumed by warp s % nw.  nw <= ns keeps every warp within one
+  // ring phase of the producer (a parity wait cannot see a phase two ahead).
+  const int nw = min(kConsumerWarps, a.ns);
   auto expert_ptr = [&](int entry) -> const uint8_t * {
     const int e = ent[entry];
     return e == E ? a.shared : a.experts + (size_t)e * G.expert_bytes;
@@ -344,74 +476,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   }
 
   // ---------------- consumers, phase C: gate/up + SwiGLU ----------------
-  // B fragments read the tokens from shared memory: scale the k pair (4c+2,
-  // 4c+3) of every 4 by 1/4 in place (exact) and negate the correction sums.
-  for (int i = tid; i < T * (H / 4); i += kConsumers) {
-    uint32_t *p2 = reinterpret_cast<uint32_t *>(xs + (i / (H / 4)) * xstride + 4 * (i % (H / 4)) + 2);
-    *p2 = bf16x2_quarter(*p2);
-  }
-  for (int i = tid; i < (H / 32) * kMaxTok; i += kConsumers) corr[i] = (i % kMaxTok) < T ? -corr[i] : 0.f;
-  named_bar(kBarConsumers, kConsumers);
-
-  const uint16_t *xrow = xs + (g < T ? g : 0) * xstride + 4 * c;
-  const bool row_ok = g < T;
-  for (int s_idx = warp; s_idx < n_gu_st; s_idx += kConsumerWarps) {
+  for (int s_idx = warp; warp < nw && s_idx < n_gu_st; s_idx += nw) {
     const int slot = s_idx % a.ns;
     bounded_wait(&full[slot], (s_idx / a.ns) & 1);
     const uint8_t *st = ring + (size_t)slot * a.stage_bytes;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int grp = 0; grp < G.gu_groups; ++grp) {
-      // one block group: 4 independent block tiles, staged load -> decode -> MMA -> scale
-      const uint8_t *gp = st + (size_t)grp * kGroupBytes;
-      const uint4 cw = lds128(gp + lane * 16);
-      const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
-      const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
-      const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
-      uint2 b0[4], b1[4];
-      float2 nc[4];
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        const int b = grp * 4 + blk;
-        b0[blk] = *reinterpret_cast<const uint2 *>(xrow + 32 * b);
-        b1[blk] = *reinterpret_cast<const uint2 *>(xrow + 32 * b + 16);
-        if (!row_ok) b0[blk] = b1[blk] = make_uint2(0u, 0u);
-        nc[blk] = *reinterpret_cast<const float2 *>(corr + b * kMaxTok + 2 * c);
-      }
-      uint32_t p[4][8];
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) decode_q2_biased(cws[blk], p[blk]);
-      float d[4][4];
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        const uint32_t a0[4] = {p[blk][0], p[blk][1], p[blk][2], p[blk][3]};
-        const float cin[4] = {nc[blk].x, nc[blk].y, nc[blk].x, nc[blk].y};
-        mma_bf16_16816(d[blk], a0, b0[blk].x, b0[blk].y, cin);
-      }
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        const uint32_t a1[4] = {p[blk][4], p[blk][5], p[blk][6], p[blk][7]};
-        mma_bf16_16816(d[blk], a1, b1[blk].x, b1[blk].y, d[blk]);
-      }
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
-        acc[0] = fmaf(s2.x, d[blk][0], acc[0]);
-        acc[1] = fmaf(s2.x, d[blk][1], acc[1]);
-        acc[2] = fmaf(s2.y, d[blk][2], acc[2]);
-        acc[3] = fmaf(s2.y, d[blk][3], acc[3]);
-      }
-    }
+    float acc[2][4];
+    if (nq == 1)
+      unit_gemv<1>(st, G.gu_groups, xb, corr, lane, acc);
+    else
+      unit_gemv<2>(st, G.gu_groups, xb, corr, lane, acc);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
     const int id = g0 + s_idx;
     const int entry = id / G.gu_units, u = id % G.gu_units;
     const int i = 8 * u + g;  // tile rows g (gate) and g+8 (up) share intermediate row i
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int n = 2 * c + half;
-      if (n < T) {
+    for (int qd = 0; qd < 2; ++qd) {
+      const int n = 4 * qd + c;  // this lane's token
+      if (qd < nq && n < T) {
         const int j = tokj[entry * kMaxTok + n];
-        if (j >= 0) a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(acc[half]) * acc[2 + half]);
+        const float gate = (acc[qd][0] + acc[qd][1]) * xsc[n], up = (acc[qd][2] + acc[qd][3]) * xsc[n];
+        if (j >= 0) a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(gate) * up);
       }
     }
   }
@@ -443,68 +528,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     }
   }
   named_bar(kBarConsumers, kConsumers);
-  for (int i = tid; i < n_hc * kMaxTok * (I / 8); i += kConsumers) {
-    const int he = i / (kMaxTok * (I / 8)), r = i % (kMaxTok * (I / 8));
+  for (int i = tid; i < n_hc * T * (I / 8); i += kConsumers) {
+    const int he = i / (T * (I / 8)), r = i % (T * (I / 8));
     const int t = r / (I / 8), c8 = r % (I / 8);
-    const int j = t < T ? tokj[(e_lo + he) * kMaxTok + t] : -1;
+    const int j = tokj[(e_lo + he) * kMaxTok + t];
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (j >= 0) v = __ldcg(reinterpret_cast<const uint4 *>(a.h + ((size_t)t * (K + 1) + j) * I + c8 * 8));
-    *reinterpret_cast<uint4 *>(hc + (he * kMaxTok + t) * hstride + c8 * 8) = v;
+    *reinterpret_cast<uint4 *>(hc + (he * T + t) * hstride + c8 * 8) = v;
   }
   named_bar(kBarConsumers, kConsumers);
+  for (int he = 0; he < n_hc; ++he)
+    build_b_fragments(hc + he * T * hstride, hstride, I, T, nq, hb + he * nq * (kMaxI / 32) * 32,
+                      hcorr + he * (kMaxI / 32) * kMaxTok, hsc + he * kMaxTok, misc + 8, warp, lane, tid);
 
-  for (int s_idx = n_gu_st + ((warp - n_gu_st % kConsumerWarps + kConsumerWarps) % kConsumerWarps); s_idx < n_st;
-       s_idx += kConsumerWarps) {
+  for (int s_idx = n_gu_st + ((warp - n_gu_st % nw + nw) % nw); warp < nw && s_idx < n_st; s_idx += nw) {
     const int sd = s_idx - n_gu_st;
     const int slot = s_idx % a.ns;
     bounded_wait(&full[slot], (s_idx / a.ns) & 1);
     const uint8_t *st = ring + (size_t)slot * a.stage_bytes;
     const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
     for (int q = q0; q < q1; ++q) {
-      const int entry = q / G.dn_units, tile = q % G.dn_units;
-      const uint16_t *hrow = hc + ((entry - e_lo) * kMaxTok + g) * hstride + 4 * c;
+      const int entry = q / G.dn_units, tile = q % G.dn_units, he = entry - e_lo;
       const uint8_t *pp_st = st + (size_t)(q - q0) * G.dn_unit_bytes;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int grp = 0; grp < 4; ++grp) {
-        const uint8_t *gp = pp_st + (size_t)grp * kGroupBytes;
-        const uint4 cw = lds128(gp + lane * 16);
-        const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
-        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
-        const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
-        uint2 b0[4], b1[4];
+      const uint2 *hbe = hb + he * nq * (kMaxI / 32) * 32;
+      const float *hce = hcorr + he * (kMaxI / 32) * kMaxTok;
+      float acc[2][4];
+      if (nq == 1)
+        unit_gemv<1>(pp_st, G.dn_groups, hbe, hce, lane, acc);
+      else
+        unit_gemv<2>(pp_st, G.dn_groups, hbe, hce, lane, acc);
+      // partial tile layout: lane (g, c) -> {row g tok c, row g+8 tok c, row g tok c+4, row g+8 tok c+4}
+      float o4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          const int b = grp * 4 + blk;
-          b0[blk] = *reinterpret_cast<const uint2 *>(hrow + 32 * b);
-          b1[blk] = *reinterpret_cast<const uint2 *>(hrow + 32 * b + 16);
-        }
-        uint32_t p[4][8];
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) decode_q2_exact(cws[blk], p[blk]);
-        float d[4][4];
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          const uint32_t a0[4] = {p[blk][0], p[blk][1], p[blk][2], p[blk][3]};
-          const float z[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_bf16_16816(d[blk], a0, b0[blk].x, b0[blk].y, z);
-        }
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          const uint32_t a1[4] = {p[blk][4], p[blk][5], p[blk][6], p[blk][7]};
-          mma_bf16_16816(d[blk], a1, b1[blk].x, b1[blk].y, d[blk]);
-        }
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
-          acc[0] = fmaf(s2.x, d[blk][0], acc[0]);
-          acc[1] = fmaf(s2.x, d[blk][1], acc[1]);
-          acc[2] = fmaf(s2.y, d[blk][2], acc[2]);
-          acc[3] = fmaf(s2.y, d[blk][3], acc[3]);
-        }
+      for (int qd = 0; qd < 2; ++qd) {
+        if (qd >= nq) break;
+        const int n = 4 * qd + c;
+        const float f = hsc[he * kMaxTok + n] * tokw[entry * kMaxTok + n];
+        o4[2 * qd] = (acc[qd][0] + acc[qd][1]) * f;
+        o4[2 * qd + 1] = (acc[qd][2] + acc[qd][3]) * f;
       }
-      const float w0 = tokw[entry * kMaxTok + 2 * c], w1 = tokw[entry * kMaxTok + 2 * c + 1];
       float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
-      *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1);
+      *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
@@ -550,11 +614,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     }
     const int r0 = 16 * tile + g;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int n = 2 * c + half;
+    for (int qd = 0; qd < 2; ++qd) {
+      const int n = 4 * qd + c;
       if (n < T) {
-        a.out[(size_t)n * H + r0] = float_to_bf16_bits(o[half]);
-        a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 + half]);
+        a.out[(size_t)n * H + r0] = float_to_bf16_bits(o[2 * qd]);
+        a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 * qd + 1]);
       }
     }
   }

@@ -182,9 +182,10 @@ moe_status moe_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_nor
 /* ---- profiling aid ------------------------------------------------------------------
  * While kernel_id >= 0, every later call made by this host thread records the
  * CUDA event `before` (a cudaEvent_t created by the caller) on its stream just
- * before it launches kernel `kernel_id`, and `after` just after, as external
- * event records, so they also become nodes of a CUDA graph being captured.
- * kernel_id < 0 turns this off.  The setting is per host thread.  The kernel
+ * before it launches kernel `kernel_id`, and `after` just after.  While the
+ * stream is being captured into a CUDA graph the records are external event
+ * records, so they become nodes of the graph; otherwise they are ordinary
+ * records.  kernel_id < 0 turns this off.  The setting is per host thread.  The kernel
  * ids below name the library's kernels and may change between versions. */
 enum {
   MOE_KERNEL_ROUTER_LOGITS = 0,
@@ -196,7 +197,9 @@ enum {
   MOE_KERNEL_DOWN = 6,
   MOE_KERNEL_COMBINE = 7,
   MOE_KERNEL_DECODE_FUSED = 8,
-  MOE_KERNEL_GATHER = 9
+  MOE_KERNEL_GATHER = 9,
+  MOE_KERNEL_FRAG_X = 10,
+  MOE_KERNEL_FRAG_H = 11
 };
 moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after);
 
