@@ -2,10 +2,10 @@
 // cooperatively launched kernel (sm_100a).  One CTA per SM: 14 consumer
 // warps and 1 producer warp.
 //
-//  A  The producer bulk-copies (TMA engine) the tokens and this CTA's router
-//     rows into shared memory and prefetches its slice of the shared expert
-//     into L2.  Consumers compute the router rows (4 warps per row, one
-//     quarter of K each) and the correction sums of the biased decode.
+//  A  The producer warp copies (cp.async, 16 B per lane) the tokens and this
+//     CTA's router rows into shared memory and prefetches its slice of the
+//     shared expert into L2.  Consumers compute the router rows (2 warps per row, one
+//     half of K each) and the correction sums of the biased decode.
 //     -- grid barrier: all logits written --
 //  B  Every CTA selects the top-k of every token (threshold + rank, one warp
 //     per token) and builds the same sorted list of touched experts plus the
@@ -42,7 +42,7 @@ namespace {
 
 constexpr int kConsumerWarps = 14;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
+constexpr int kThreads = kConsumers;  // every warp computes and streams its own stages
 constexpr int kMaxTok = 8;
 constexpr int kMaxSel = 128;              // T * top_k
 constexpr int kMaxEntries = kMaxSel + 1;  // touched experts + shared
@@ -67,12 +67,13 @@ struct DecodeArgs {
   float *w_out;        // optional [T][k]
   uint16_t *out;       // [T][H]
   uint32_t *status;
-  int ns;              // ring stages
+  int ns;              // ring stages: nw warps x (ns / nw) private slots each
+  int nw;              // warps that stream and compute expert stages
   uint32_t stage_bytes;
 };
 
 struct SmemLayout {
-  uint32_t bars, xs, corr, xb, xsc, hb, hcorr, hsc, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc,
+  uint32_t xs, corr, xb, xsc, hb, hcorr, hsc, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc,
       ring, total;
 };
 
@@ -84,8 +85,6 @@ __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v
 __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes) {
   SmemLayout L;
   uint32_t o = 0;
-  L.bars = o;  // full[ns], empty[ns], rbar, xbar
-  o = align_to(o + 8u * (2 * ns + 2), 16);
   // xs: the tokens (bf16 rows, phase A).  The same bytes hold the h fragments of phase D.
   const uint32_t hb_bytes = 2u * token_quads(T) * (kMaxI / 32) * 256;
   const uint32_t hcorr_bytes = 2u * (kMaxI / 32) * kMaxTok * 4;
@@ -101,8 +100,8 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   o = align_to(o + (uint32_t)token_quads(T) * (H / 32) * 256, 16);
   L.xsc = o;  // [8] 2^(9 - s_t): undoes the token scale and the 2^-9 of the A bytes
   o += kMaxTok * 4;
-  L.rpart = o;  // [rows per pass <= 4][8 tokens][4 quarters]
-  o += 4 * kMaxTok * 4 * 4;
+  L.rpart = o;  // [rows per pass][8 tokens][router parts]
+  o += (kConsumerWarps / kRouterParts) * kMaxTok * kRouterParts * 4;
   L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
   o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
   L.sel_idx = o;
@@ -254,10 +253,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const PackedGeom &G = a.G;
   const int T = a.T, E = a.E, K = a.k, H = G.H, I = G.I;
   const SmemLayout L = smem_layout(T, H, a.ns, a.stage_bytes);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
-  uint64_t *empty = full + a.ns;
-  uint64_t *rbar = empty + a.ns;
-  uint64_t *xbar = rbar + 1;
   uint16_t *xs = reinterpret_cast<uint16_t *>(smem + L.xs);
   float *corr = reinterpret_cast<float *>(smem + L.corr);
   uint2 *xb = reinterpret_cast<uint2 *>(smem + L.xb);
@@ -280,70 +275,52 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   uint32_t *ready = a.tile_cnt + G.dn_units;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool is_producer = warp == kConsumerWarps;
   const int g = lane >> 2, c = lane & 3;
   const int xstride = H + 16;
   const int n_rrows = E > (int)blockIdx.x ? (E - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   float *wr_s = reinterpret_cast<float *>(ring);  // router rows live in the ring until phase C
 
-  // A wait that hits its limit marks the CTA aborted; later waits are skipped
-  // so every warp keeps the same control flow and the kernel ends in bounded
-  // time with the timeout bit set.
-  auto bounded_wait = [&](uint64_t *bar, uint32_t parity) {
-    if (*reinterpret_cast<volatile int *>(&misc[1])) return;
-    if (!mbar_wait(bar, parity)) {
-      set_status(a.status, kStatusTimeout);
-      misc[1] = 1;
-    }
-  };
-
   // ---------------- phase A: set-up, router ----------------
-  if (tid == 0) {
-    for (int i = 0; i < a.ns; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);  // each stage is consumed by one warp
-    }
-    mbar_init(rbar, 1);
-    mbar_init(xbar, 1);
-    mbar_fence_init();
-    for (int i = 0; i < 8; ++i) misc[i] = 0;
+  if (tid == 0)
+    for (int i = 0; i < 16; ++i) misc[i] = 0;
+  // The tokens, then this CTA's router rows: cp.async pieces from every thread
+  // (two commit groups), and an L2 prefetch of this CTA's slice of the shared expert.
+  for (int i = tid; i < T * (H / 8); i += kConsumers) {
+    const int t = i / (H / 8), c8 = i % (H / 8);
+    cp_async16(xs + t * xstride + c8 * 8, a.x + (size_t)t * H + c8 * 8);
   }
-  __syncthreads();
-
-  if (is_producer) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(xbar, (uint32_t)(T * H * 2));
-      for (int t = 0; t < T; ++t) bulk_g2s(xs + t * xstride, a.x + (size_t)t * H, (uint32_t)(H * 2), xbar);
-      if (n_rrows > 0) {
-        mbar_arrive_expect_tx(rbar, (uint32_t)(n_rrows * H * 4));
-        for (int r = 0; r < n_rrows; ++r)
-          bulk_g2s(wr_s + (size_t)r * H, a.Wr + (size_t)(blockIdx.x + (size_t)gridDim.x * r) * H, (uint32_t)(H * 4),
-                   rbar);
-      }
-      const size_t per = ((G.expert_bytes + gridDim.x - 1) / gridDim.x + 15) & ~(size_t)15;
-      const size_t off = per * blockIdx.x;
-      if (off < G.expert_bytes) {
-        const size_t n = min(per, G.expert_bytes - off);
-        for (size_t o = 0; o < n; o += 32768)
-          bulk_prefetch_l2(a.shared + off + o, (uint32_t)min((size_t)32768, n - o));
-      }
+  cp_async_commit();
+  for (int i = tid; i < n_rrows * (H / 4); i += kConsumers) {
+    const int r = i / (H / 4), c4 = i % (H / 4);
+    cp_async16(wr_s + (size_t)r * H + c4 * 4, a.Wr + (size_t)(blockIdx.x + (size_t)gridDim.x * r) * H + c4 * 4);
+  }
+  cp_async_commit();
+  if (tid == 0) {
+    const size_t per = ((G.expert_bytes + gridDim.x - 1) / gridDim.x + 15) & ~(size_t)15;
+    const size_t off = per * blockIdx.x;
+    if (off < G.expert_bytes) {
+      const size_t n = min(per, G.expert_bytes - off);
+      for (size_t o = 0; o < n; o += 32768) bulk_prefetch_l2(a.shared + off + o, (uint32_t)min((size_t)32768, n - o));
     }
-  } else {
+  }
+  {
     if (blockIdx.x == 0)
       for (int i = tid; i < G.dn_units + kMaxEntries; i += kConsumers) a.tile_cnt[i] = 0u;
-    bounded_wait(xbar, 0);
+    cp_async_wait_group<1>();  // this thread's token pieces have landed
+    named_bar(kBarConsumers, kConsumers);
     // Tokens as e4m3 B fragments: per-token power-of-two scale, two split terms.
     build_b_fragments(xs, xstride, H, T, nq, xb, corr, xsc, misc + 8, warp, lane, tid);
-    bounded_wait(rbar, 0);
-    constexpr int kRowsPerPass = kConsumerWarps / 4;  // 4 warps (quarters) per router row
+    cp_async_wait_group<0>();  // router rows
+    named_bar(kBarConsumers, kConsumers);
+    constexpr int kRowsPerPass = kConsumerWarps / kRouterParts;  // one warp per router row part
     for (int r0 = 0; r0 < n_rrows; r0 += kRowsPerPass) {
-      const int r = r0 + (warp >> 2), q = warp & 3;
+      const int r = r0 + warp / kRouterParts, q = warp % kRouterParts;
       if (r < n_rrows) {
         float acc[8];
-        router_quarter<true>(xs, xstride, T, wr_s + (size_t)r * H, H, q, lane, acc);
+        router_part<true>(xs, xstride, T, wr_s + (size_t)r * H, H, q, lane, acc);
         if (lane == 0) {
 #pragma unroll
-          for (int t = 0; t < 8; ++t) rpart[((r - r0) * kMaxTok + t) * 4 + q] = acc[t];
+          for (int t = 0; t < 8; ++t) rpart[((r - r0) * kMaxTok + t) * kRouterParts + q] = acc[t];
         }
       }
       named_bar(kBarConsumers, kConsumers);
@@ -351,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         const int rr = tid / T, t = tid % T;
         if (r0 + rr < n_rrows) {
           const int e = blockIdx.x + gridDim.x * (r0 + rr);
-          a.logits[(size_t)t * E + e] = router_combine(rpart + (rr * kMaxTok + t) * 4, a.bias ? a.bias[e] : 0.f);
+          a.logits[(size_t)t * E + e] =
+              router_combine(rpart + (rr * kMaxTok + t) * kRouterParts, a.bias ? a.bias[e] : 0.f);
         }
       }
       named_bar(kBarConsumers, kConsumers);
@@ -359,14 +337,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     grid_barrier(&a.gbar[0], &a.gbar[1], kBarConsumers, kConsumers, tid == 0, a.status, &misc[2]);
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
+    // All logits into shared memory first (one coalesced pass through L2), then one warp per token.
+    float *lg = reinterpret_cast<float *>(ring);  // the ring is free until the stages start
+    for (int i = tid; i < T * E / 4; i += kConsumers)
+      reinterpret_cast<float4 *>(lg)[i] = ldg_cg_f4(a.logits + 4 * (size_t)i);
+    for (int i = (T * E / 4) * 4 + tid; i < T * E; i += kConsumers) lg[i] = __ldcg(a.logits + i);
+    named_bar(kBarConsumers, kConsumers);
     if (warp < T) {
       int e;
       float wt;
       uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
       if (E <= 512)
-        warp_topk_fast<16>(a.logits + (size_t)warp * E, E, K, lane, scratch, e, wt);
+        warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
       else
-        warp_topk_fast<32>(a.logits + (size_t)warp * E, E, K, lane, scratch, e, wt);
+        warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
       if (lane < K) {
         sel_idx[warp * K + lane] = e;
         sel_w[warp * K + lane] = wt;
@@ -420,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       }
     }
   }
-  __syncthreads();  // the list is visible to the producer as well
+  __syncthreads();  // the list is visible to every warp
 
   const int nent = misc[0];
   const int n_gu = nent * G.gu_units, n_dn = nent * G.dn_units;
@@ -432,61 +416,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const int n_gu_st = g1 - g0;
   const int n_dn_st = (d1 - d0 + pps - 1) / pps;
   const int n_st = n_gu_st + n_dn_st;
-  // Stage s is consumed by warp s % nw.  nw <= ns keeps every warp within one
-  // ring phase of the producer (a parity wait cannot see a phase two ahead).
-  const int nw = min(kConsumerWarps, a.ns);
+  // Stage s belongs to warp s % nw, which copies it (cp.async) into one of its
+  // own spw ring slots, waits for its own copies, computes it and refills the
+  // slot with its stage s + spw * nw.  No other warp touches the slot.
+  const int nw = a.nw, spw = a.ns / a.nw;
   auto expert_ptr = [&](int entry) -> const uint8_t * {
     const int e = ent[entry];
     return e == E ? a.shared : a.experts + (size_t)e * G.expert_bytes;
   };
-
-  if (is_producer) {
-    // ---------------- producer: stream this CTA's units into the ring ----------------
-    if (lane == 0) {
-      int issued = 0;
-      for (int s = 0; s < n_st; ++s) {
-        const int slot = s % a.ns;
-        if (*reinterpret_cast<volatile int *>(&misc[1]) || !mbar_wait(&empty[slot], ((s / a.ns) & 1) ^ 1)) {
-          set_status(a.status, kStatusTimeout);
-          misc[1] = 1;
-          break;
-        }
-        uint8_t *dst = ring + (size_t)slot * a.stage_bytes;
-        if (s < n_gu_st) {
-          const int id = g0 + s;
-          const uint8_t *src = expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes;
-          mbar_arrive_expect_tx(&full[slot], (uint32_t)G.gu_unit_bytes);
-          bulk_g2s(dst, src, (uint32_t)G.gu_unit_bytes, &full[slot]);
-        } else {
-          const int q0 = d0 + (s - n_gu_st) * pps, q1 = min(d1, q0 + pps);
-          mbar_arrive_expect_tx(&full[slot], (uint32_t)((q1 - q0) * G.dn_unit_bytes));
-          for (int q = q0; q < q1; ++q) {
-            const uint8_t *src =
-                expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes;
-            bulk_g2s(dst + (size_t)(q - q0) * G.dn_unit_bytes, src, (uint32_t)G.dn_unit_bytes, &full[slot]);
-          }
-        }
-        issued = s + 1;
+  auto stage_ptr = [&](int s) { return ring + (size_t)(warp * spw + (s / nw) % spw) * a.stage_bytes; };
+  auto issue_stage = [&](int s) {  // one commit group per call, empty past the last stage
+    if (s < n_st) {
+      uint8_t *dst = stage_ptr(s);
+      if (s < n_gu_st) {
+        const int id = g0 + s;
+        warp_cp_async(dst, expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes,
+                      (uint32_t)G.gu_unit_bytes, lane);
+      } else {
+        const int q0 = d0 + (s - n_gu_st) * pps, q1 = min(d1, q0 + pps);
+        for (int q = q0; q < q1; ++q)
+          warp_cp_async(dst + (size_t)(q - q0) * G.dn_unit_bytes,
+                        expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes,
+                        (uint32_t)G.dn_unit_bytes, lane);
       }
-      // Before the CTA may exit, every copy this thread issued must have landed.
-      for (int s = max(0, issued - a.ns); s < issued; ++s)
-        if (!mbar_wait(&full[s % a.ns], (s / a.ns) & 1)) set_status(a.status, kStatusTimeout);
     }
-    return;
-  }
+    cp_async_commit();
+  };
+  auto wait_stage = [&]() {  // the oldest of this warp's spw outstanding stages has landed
+    if (spw == 1)
+      cp_async_wait_group<0>();
+    else
+      cp_async_wait_group<1>();
+    __syncwarp();
+  };
+  if (warp < nw)
+    for (int j = 0; j < spw; ++j) issue_stage(warp + j * nw);
 
   // ---------------- consumers, phase C: gate/up + SwiGLU ----------------
   for (int s_idx = warp; warp < nw && s_idx < n_gu_st; s_idx += nw) {
-    const int slot = s_idx % a.ns;
-    bounded_wait(&full[slot], (s_idx / a.ns) & 1);
-    const uint8_t *st = ring + (size_t)slot * a.stage_bytes;
+    wait_stage();
+    const uint8_t *st = stage_ptr(s_idx);
     float acc[2][4];
     if (nq == 1)
       unit_gemv<1>(st, G.gu_groups, xb, corr, lane, acc);
     else
       unit_gemv<2>(st, G.gu_groups, xb, corr, lane, acc);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
+    issue_stage(s_idx + spw * nw);
     const int id = g0 + s_idx;
     const int entry = id / G.gu_units, u = id % G.gu_units;
     const int i = 8 * u + g;  // tile rows g (gate) and g+8 (up) share intermediate row i
@@ -543,9 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
 
   for (int s_idx = n_gu_st + ((warp - n_gu_st % nw + nw) % nw); warp < nw && s_idx < n_st; s_idx += nw) {
     const int sd = s_idx - n_gu_st;
-    const int slot = s_idx % a.ns;
-    bounded_wait(&full[slot], (s_idx / a.ns) & 1);
-    const uint8_t *st = ring + (size_t)slot * a.stage_bytes;
+    wait_stage();
+    const uint8_t *st = stage_ptr(s_idx);
     const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
     for (int q = q0; q < q1; ++q) {
       const int entry = q / G.dn_units, tile = q % G.dn_units, he = entry - e_lo;
@@ -571,8 +546,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
+    issue_stage(s_idx + spw * nw);
   }
+  cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
 
   // Count this CTA's contributions per output tile (one fence per writer
   // warp); the last contributor of a tile sums its partials in expert order.
@@ -652,9 +628,10 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const uint32_t stage_bytes = (uint32_t)max(G.gu_unit_bytes, 4 * G.dn_unit_bytes);
   const SmemLayout L0 = smem_layout(T, G.H, 0, stage_bytes);
-  int ns = (int)((max_smem - (int)L0.ring - 128) / (int)(stage_bytes + 16));
-  ns = min(ns, 32);
-  if (ns < 2) return cudaErrorInvalidConfiguration;
+  const int slots = (int)((max_smem - (int)L0.ring - 128) / (int)stage_bytes);
+  if (slots < 1) return cudaErrorInvalidConfiguration;
+  const int nw = min(kConsumerWarps, slots);        // warps streaming and computing stages
+  const int ns = nw * min(2, slots / nw);           // 1 or 2 private slots per warp
   const SmemLayout L = smem_layout(T, G.H, ns, stage_bytes);
   if (L.total > (uint32_t)max_smem) return cudaErrorInvalidConfiguration;
   // the per-CTA down range must fit the 128-entry completed-tile list
@@ -662,6 +639,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   if ((max_entries * G.dn_units + n_sm - 1) / n_sm > kMaxSel) return cudaErrorInvalidConfiguration;
   const int rrows = (d.n_experts + n_sm - 1) / n_sm;  // router rows per CTA, staged in the ring
   if ((size_t)rrows * d.hidden * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;
+  if ((size_t)T * d.n_experts * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;  // logits
 
   DecodeArgs a{};
   a.x = x;
@@ -683,6 +661,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   a.out = out;
   a.status = ws.status;
   a.ns = ns;
+  a.nw = nw;
   a.stage_bytes = stage_bytes;
 
   void (*kern)(DecodeArgs) = decode_fused_kernel;

@@ -10,12 +10,12 @@
 //   frag_prep (h)  the same for every h row;
 //   grouped<1>     down -> fp32 expert output per sorted position, summed by
 //                  the combine kernel.
-// grouped<MODE> runs one persistent CTA per SM with 16 consumer warps and one
-// producer warp.  A work item is a token tile (<= 32 sorted positions of one
+// grouped<MODE> runs one persistent CTA per SM with 16 warps.  A work item is a token tile (<= 32 sorted positions of one
 // expert) times a group of 16 units (16-row tiles of the projection).  For
-// every 128-wide K chunk the producer bulk-copies (TMA engine) the 16 units'
-// packed codes and scales of that chunk (640 B each) and each token's 272-byte
-// chunk record into a shared-memory stage; consumer warp u runs unit
+// every 128-wide K chunk the warps copy (cp.async, 16 B per lane; warp u takes
+// unit u and every 16th token) the 16 units' packed codes and scales of that
+// chunk (640 B each) and each token's 272-byte chunk record into a
+// shared-memory stage, ns stages ahead of use; warp u runs unit
 // u's 4 block tiles against every token quad of the tile (one m16n8k32 MMA per
 // block and quad, accumulator started at the block correction), scales each
 // block result by its fp16 d and keeps the sums in registers across chunks.
@@ -29,7 +29,7 @@ namespace moe {
 namespace {
 
 constexpr int kGW = 16;                   // consumer warps = units per work item
-constexpr int kGThreads = (kGW + 1) * 32;
+constexpr int kGThreads = kGW * 32;
 constexpr int kTileTok = 32;              // sorted positions per work item (8 token quads)
 constexpr int kChunkRec = 4 * 64 + 16;     // per token and K chunk: 4 block records + 4 corrections
 constexpr int kTokStride = 320;            // shared-memory stride of a token's chunk record (bank spread)
@@ -91,7 +91,7 @@ __device__ __forceinline__ void chunk_mma(const uint8_t *st, int u, int lane, fl
 }
 
 template <int MODE>  // 0: gate/up + SwiGLU -> h; 1: down -> y
-__global__ void __maxnreg__(96) grouped_kernel(const GArgs a) {  // 17 warps: 5 share one SM sub-partition's 16K registers
+__global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)a.ns * kStageBytes);
   uint64_t *empty = full + a.ns;
@@ -101,56 +101,39 @@ __global__ void __maxnreg__(96) grouped_kernel(const GArgs a) {  // 17 warps: 5 
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.ns; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kGW);
+      mbar_init(&full[i], kGThreads);  // one cp.async arrival per thread
+      mbar_init(&empty[i], kGW);       // one arrival per warp once it has read the stage
     }
     *abort_flag = 0;
     mbar_fence_init();
   }
   __syncthreads();
 
-  if (warp == kGW) {
-    // ---- producer ----
-    int cnt = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
-      const int4 tile = a.tiles[w / a.ugroups];
-      const int u0 = (w % a.ugroups) * kGW, nu = min(kGW, a.units - u0);
-      const uint8_t *eb = (tile.x == a.E ? a.shared : a.experts + (size_t)tile.x * a.G.expert_bytes) + a.sec_off +
-                          (size_t)u0 * a.unit_bytes;
-      const int ntok = tile.z;
-      const int row = lane < ntok ? (a.row_of_pos ? a.row_of_pos[tile.y + lane] : tile.y + lane) : -1;
-      const uint8_t *src_b = row >= 0 ? a.frag + (size_t)row * a.kchunks * kChunkRec : nullptr;
-      for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
-        const int s = cnt % a.ns;
-        if (lane == 0) {
-          ok = !*abort_flag && mbar_wait(&empty[s], ((cnt / a.ns) & 1) ^ 1);
-          if (ok)
-            mbar_arrive_expect_tx(&full[s], (uint32_t)(nu * kGroupBytes + ntok * kChunkRec));
-          else {
-            set_status(a.status, kStatusTimeout);
-            *abort_flag = 1;
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
-        uint8_t *st = smem + (size_t)s * kStageBytes;
-        if (lane < nu)
-          bulk_g2s(st + lane * kGroupBytes, eb + (size_t)lane * a.unit_bytes + (size_t)kc * kGroupBytes,
-                   kGroupBytes, &full[s]);
-        if (row >= 0)
-          bulk_g2s(st + kStageA + lane * kTokStride, src_b + (size_t)kc * kChunkRec, kChunkRec, &full[s]);
-      }
-    }
-    // every copy issued must land before the CTA may exit
-    if (lane == 0)
-      for (int c2 = max(0, cnt - a.ns); c2 < cnt; ++c2)
-        if (!mbar_wait(&full[c2 % a.ns], (c2 / a.ns) & 1)) set_status(a.status, kStatusTimeout);
-    return;
-  }
-
-  // ---- consumers: warp u owns unit u of the item's group ----
   const int u = warp, g = lane >> 2, c = lane & 3;
+  const int n_stages = ((n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * a.kchunks;
+  // Every warp copies its share of stage q (this CTA's q-th K chunk): unit u's
+  // 640-byte piece and the chunk records of tokens u and u + 16; then each
+  // thread arrives on the stage's full barrier once its copies have landed.
+  auto issue = [&](int q) {
+    const int w = (int)blockIdx.x + (q / a.kchunks) * (int)gridDim.x, kc = q % a.kchunks;
+    const int4 tile = a.tiles[w / a.ugroups];
+    const int u0 = (w % a.ugroups) * kGW, nu = min(kGW, a.units - u0);
+    uint8_t *st = smem + (size_t)(q % a.ns) * kStageBytes;
+    if (u < nu) {
+      const uint8_t *src = (tile.x == a.E ? a.shared : a.experts + (size_t)tile.x * a.G.expert_bytes) + a.sec_off +
+                           (size_t)(u0 + u) * a.unit_bytes + (size_t)kc * kGroupBytes;
+      for (int i = lane; i < kGroupBytes / 16; i += 32) cp_async16(st + u * kGroupBytes + i * 16, src + i * 16);
+    }
+    for (int tk = u; tk < tile.z; tk += kGW) {
+      const int r = a.row_of_pos ? a.row_of_pos[tile.y + tk] : tile.y + tk;
+      if (lane < kChunkRec / 16)
+        cp_async16(st + kStageA + tk * kTokStride + lane * 16,
+                   a.frag + ((size_t)r * a.kchunks + kc) * kChunkRec + lane * 16);
+    }
+    cp_async_arrive(&full[q % a.ns]);
+  };
+  for (int q = 0; q < min(a.ns, n_stages); ++q) issue(q);
+
   int cnt = 0;
   for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
     const int4 tile = a.tiles[w / a.ugroups];
@@ -183,6 +166,14 @@ __global__ void __maxnreg__(96) grouped_kernel(const GArgs a) {  // 17 warps: 5 
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
+      // refill this slot with stage cnt + ns once every warp has read it
+      if (cnt + a.ns < n_stages) {
+        if (!*abort_flag && !mbar_wait(&empty[s], (cnt / a.ns) & 1)) {
+          set_status(a.status, kStatusTimeout);
+          *abort_flag = 1;
+        }
+        if (!*abort_flag) issue(cnt + a.ns);
+      }
     }
     if (!active || *abort_flag) continue;
 #pragma unroll
@@ -203,6 +194,7 @@ __global__ void __maxnreg__(96) grouped_kernel(const GArgs a) {  // 17 warps: 5 
       }
     }
   }
+  cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
 }
 
 // One warp per row of v ([rows][K] bf16): the row's unscale factor 2^(9 - s),

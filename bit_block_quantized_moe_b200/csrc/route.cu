@@ -9,6 +9,7 @@
 
 #include "kernels.cuh"
 #include "router.cuh"
+#include "sync.cuh"
 
 namespace moe {
 
@@ -119,19 +120,19 @@ __device__ __forceinline__ void clear_range(uint32_t *p, size_t n) {
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
 }
 
-// Few tokens (T <= 8): one CTA of 4 warps per expert row, warp q summing the
-// row's quarter q (router_quarter), combined in quarter order.
-__global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t *__restrict__ x,
-                                                                   const float *__restrict__ Wr,
-                                                                   const float *__restrict__ bias, int T, int H,
-                                                                   int E, float *__restrict__ logits,
-                                                                   uint32_t *zero_p, size_t zero_n) {
+// Few tokens (T <= 8): one CTA of 2 warps per expert row, warp h summing the
+// row's half h (router_part), combined in half order.
+__global__ void __launch_bounds__(64) router_logits_small_kernel(const uint16_t *__restrict__ x,
+                                                                  const float *__restrict__ Wr,
+                                                                  const float *__restrict__ bias, int T, int H,
+                                                                  int E, float *__restrict__ logits,
+                                                                  uint32_t *zero_p, size_t zero_n) {
   clear_range(zero_p, zero_n);
-  __shared__ float part[8][4];
+  __shared__ float part[8][kRouterParts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x;
   float acc[8];
-  router_quarter<false>(x, H, T, Wr + (size_t)e * H, H, warp, lane, acc);
+  router_part<false>(x, H, T, Wr + (size_t)e * H, H, warp, lane, acc);
   if (lane == 0) {
 #pragma unroll
     for (int t = 0; t < 8; ++t) part[t][warp] = acc[t];
@@ -145,8 +146,7 @@ __global__ void __launch_bounds__(128) router_logits_small_kernel(const uint16_t
 // significant bits); x is bf16 already, so every product is exact in fp32 and
 // only the fp32 accumulation rounds, as in a CUDA-core dot product.  Each
 // 256-wide K slice is accumulated in a fresh tensor-core accumulator and then
-// added to the running fp32 sum.  CTA tile: 64 experts x 64 tokens, 8 warps of
-// 16 experts x 32 tokens (m16n8k16).
+// added to the running fp32 sum.
 __device__ __forceinline__ void split3_bf16(float w, uint16_t &hi, uint16_t &mid, uint16_t &lo) {
   hi = float_to_bf16_bits(w);
   const float r1 = w - bf16_bits_to_float(hi);
@@ -155,44 +155,69 @@ __device__ __forceinline__ void split3_bf16(float w, uint16_t &hi, uint16_t &mid
   lo = float_to_bf16_bits(r2);
 }
 
-__global__ void __launch_bounds__(256) router_logits_mma_kernel(const uint16_t *__restrict__ x,
+constexpr int kRbE = 64, kRbT = 32, kRbK = 64, kRbStages = 3;  // CTA tile: experts x tokens x K step
+constexpr int kRwStride = kRbK + 8;                                // floats (bank spread for float2 reads)
+constexpr int kRxStride = kRbK + 8;                                // bf16
+constexpr int kRwBytes = kRbE * kRwStride * 4;
+constexpr int kRxBytes = kRbT * kRxStride * 2;
+constexpr int kRStageBytes = kRwBytes + kRxBytes;
+constexpr int kRouterSmem = kRbStages * kRStageBytes;
+
+__device__ __forceinline__ void cp_async16_zfill(void *dst_smem, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+// CTA tile 64 experts x 32 tokens, 4 warps of 16 experts x 32 tokens; K in
+// steps of 64 through a 3-stage cp.async pipeline (rows past E or T read as 0).
+__global__ void __launch_bounds__(128) router_logits_mma_kernel(const uint16_t *__restrict__ x,
                                                                  const float *__restrict__ Wr,
                                                                  const float *__restrict__ bias, int T, int H, int E,
                                                                  float *__restrict__ logits, uint32_t *zero_p,
                                                                  size_t zero_n) {
   clear_range(zero_p, zero_n);
-  constexpr int BK = 32, WS = BK + 4, XS = BK + 8;  // padded row strides (floats / halves)
-  __shared__ float ws[64 * WS];
-  __shared__ uint16_t xs[64 * XS];
-  const int e0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int wm = warp & 3, wn = warp >> 2;
+  extern __shared__ __align__(16) uint8_t rsm[];
+  const int e0 = blockIdx.x * kRbE, t0 = blockIdx.y * kRbT;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+  const int nk = H / kRbK;
+  auto load_stage = [&](int st, int k0) {
+    float *ws = reinterpret_cast<float *>(rsm + st * kRStageBytes);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(rsm + st * kRStageBytes + kRwBytes);
+#pragma unroll
+    for (int j = 0; j < (kRbE * kRbK / 4) / 128; ++j) {
+      const int i = tid + 128 * j, r = i / (kRbK / 4), c4 = i % (kRbK / 4);
+      const bool ok = e0 + r < E;
+      cp_async16_zfill(ws + r * kRwStride + 4 * c4, Wr + (size_t)(ok ? e0 + r : 0) * H + k0 + 4 * c4, ok);
+    }
+#pragma unroll
+    for (int j = 0; j < (kRbT * kRbK / 8) / 128; ++j) {
+      const int i = tid + 128 * j, r = i / (kRbK / 8), c8 = i % (kRbK / 8);
+      const bool ok = t0 + r < T;
+      cp_async16_zfill(xs + r * kRxStride + 8 * c8, x + (size_t)(ok ? t0 + r : 0) * H + k0 + 8 * c8, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
   float acc[4][4] = {};
   float part[4][4] = {};
-  for (int k0 = 0; k0 < H; k0 += BK) {
-    // stage 64 x 32 router weights and 64 x 32 tokens
-    for (int i = threadIdx.x; i < 64 * (BK / 4); i += 256) {
-      const int r = i / (BK / 4), c4 = i % (BK / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e0 + r < E) v = *reinterpret_cast<const float4 *>(Wr + (size_t)(e0 + r) * H + k0 + 4 * c4);
-      *reinterpret_cast<float4 *>(ws + r * WS + 4 * c4) = v;
-    }
-    for (int i = threadIdx.x; i < 64 * (BK / 8); i += 256) {
-      const int r = i / (BK / 8), c8 = i % (BK / 8);
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (t0 + r < T) v = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + r) * H + k0 + 8 * c8);
-      *reinterpret_cast<uint2 *>(xs + r * XS + 8 * c8) = make_uint2(v.x, v.y);
-      *reinterpret_cast<uint2 *>(xs + r * XS + 8 * c8 + 4) = make_uint2(v.z, v.w);
-    }
-    __syncthreads();
+  load_stage(0, 0);
+  if (nk > 1) load_stage(1, kRbK);
+  else asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int kt = 0; kt < nk; ++kt) {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();  // stage kt visible to all; stage (kt + 2) % 3 no longer read
+    if (kt + 2 < nk) load_stage((kt + 2) % kRbStages, (kt + 2) * kRbK);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    const float *ws = reinterpret_cast<const float *>(rsm + (kt % kRbStages) * kRStageBytes);
+    const uint16_t *xs = reinterpret_cast<const uint16_t *>(rsm + (kt % kRbStages) * kRStageBytes + kRwBytes);
 #pragma unroll
-    for (int kk = 0; kk < BK; kk += 16) {
-      // A fragments of the three splits: rows wm*16 + g (+8), k = kk + 2c (+1) and kk + 2c + 8 (+9)
+    for (int kk = 0; kk < kRbK; kk += 16) {
+      // A fragments of the three splits: rows 16 * warp + g (+8), k = kk + 2c (+1) and kk + 2c + 8 (+9)
       uint32_t ah[4], am[4], al[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int row = wm * 16 + g + 8 * (q & 1), col = kk + 2 * c + 8 * (q >> 1);
-        const float2 w2 = *reinterpret_cast<const float2 *>(ws + row * WS + col);
+        const int row = warp * 16 + g + 8 * (q & 1), col = kk + 2 * c + 8 * (q >> 1);
+        const float2 w2 = *reinterpret_cast<const float2 *>(ws + row * kRwStride + col);
         uint16_t h0, m0, l0, h1, m1, l1;
         split3_bf16(w2.x, h0, m0, l0);
         split3_bf16(w2.y, h1, m1, l1);
@@ -202,7 +227,7 @@ __global__ void __launch_bounds__(256) router_logits_mma_kernel(const uint16_t *
       }
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
-        const uint16_t *xr = xs + (wn * 32 + nt * 8 + g) * XS + kk + 2 * c;
+        const uint16_t *xr = xs + (nt * 8 + g) * kRxStride + kk + 2 * c;
         const uint32_t b0 = *reinterpret_cast<const uint32_t *>(xr);
         const uint32_t b1 = *reinterpret_cast<const uint32_t *>(xr + 8);
         mma_bf16_16816(part[nt], ah, b0, b1, part[nt]);
@@ -210,8 +235,7 @@ __global__ void __launch_bounds__(256) router_logits_mma_kernel(const uint16_t *
         mma_bf16_16816(part[nt], al, b0, b1, part[nt]);
       }
     }
-    __syncthreads();
-    if (((k0 + BK) & 255) == 0 || k0 + BK >= H) {  // end of a 256-wide K slice
+    if ((((kt + 1) * kRbK) & 255) == 0 || kt + 1 == nk) {  // end of a 256-wide K slice
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -221,13 +245,14 @@ __global__ void __launch_bounds__(256) router_logits_mma_kernel(const uint16_t *
         }
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   // D fragment: (row g, cols 2c, 2c+1), (row g+8, cols 2c, 2c+1); rows = experts, cols = tokens
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int e = e0 + wm * 16 + g + 8 * (q >> 1);
-      const int t = t0 + wn * 32 + nt * 8 + 2 * c + (q & 1);
+      const int e = e0 + warp * 16 + g + 8 * (q >> 1);
+      const int t = t0 + nt * 8 + 2 * c + (q & 1);
       if (e < E && t < T) logits[(size_t)t * E + e] = acc[nt][q] + (bias ? bias[e] : 0.f);
     }
 }
@@ -262,12 +287,16 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, 
   const int H = d.hidden, E = d.n_experts, k = d.top_k;
   if (T <= 8) {
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
-    router_logits_small_kernel<<<E, 128, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin, ws.zero_words);
+    router_logits_small_kernel<<<E, 32 * kRouterParts, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin, ws.zero_words);
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
   } else {
-    dim3 grid((E + 63) / 64, (T + 63) / 64);
+    dim3 grid((E + kRbE - 1) / kRbE, (T + kRbT - 1) / kRbT);
+    cudaError_t e0 = cudaFuncSetAttribute(router_logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          kRouterSmem);
+    if (e0 != cudaSuccess) return e0;
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
-    router_logits_mma_kernel<<<grid, 256, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin, ws.zero_words);
+    router_logits_mma_kernel<<<grid, 128, kRouterSmem, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin,
+                                                            ws.zero_words);
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
   }
   cudaError_t err = cudaGetLastError();

@@ -6,19 +6,20 @@
 
 namespace moe {
 
-// Router arithmetic for T <= 8 tokens.  The row is cut into 4 quarters of
-// H/4; quarter q is summed by one warp: lane l accumulates k = q*H/4 + 4l +
-// 128 i in order, then a butterfly sum.  The logit is ((p0 + p1) + p2) + p3 + b.
-// Both the routing kernel and the fused decode kernel use exactly this order,
-// so they take identical routing decisions.
+// Router arithmetic for T <= 8 tokens.  The row is cut into 2 halves of H/2;
+// half h is summed by one warp: lane l accumulates k = h*H/2 + 4l + 128 i in
+// order, then a butterfly sum.  The logit is (p0 + p1) + b.  Both the routing
+// kernel and the fused decode kernel use exactly this order, so they take
+// identical routing decisions.
+constexpr int kRouterParts = 2;
 template <bool kWrShared>
-__device__ __forceinline__ void router_quarter(const uint16_t *x, int xstride, int T, const float *wrow, int H,
-                                               int quarter, int lane, float (&acc)[8]) {
+__device__ __forceinline__ void router_part(const uint16_t *x, int xstride, int T, const float *wrow, int H,
+                                            int part, int lane, float (&acc)[8]) {
 #pragma unroll
   for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-  const int kq = H / 4;
+  const int kq = H / kRouterParts;
 #pragma unroll 4
-  for (int k = quarter * kq + lane * 4; k < (quarter + 1) * kq; k += 128) {
+  for (int k = part * kq + lane * 4; k < (part + 1) * kq; k += 128) {
     const uint4 wv = kWrShared ? *reinterpret_cast<const uint4 *>(wrow + k) : ldg_nc_v4(wrow + k);
     const float w0 = __uint_as_float(wv.x), w1 = __uint_as_float(wv.y), w2 = __uint_as_float(wv.z),
                 w3 = __uint_as_float(wv.w);
@@ -42,9 +43,7 @@ __device__ __forceinline__ void router_quarter(const uint16_t *x, int xstride, i
   }
 }
 
-__device__ __forceinline__ float router_combine(const float *part4, float b) {
-  return ((part4[0] + part4[1]) + part4[2]) + part4[3] + b;
-}
+__device__ __forceinline__ float router_combine(const float *parts, float b) { return (parts[0] + parts[1]) + b; }
 
 // fp32 softmax over the k winners held by lanes 0..k-1 (lane order = selection order).
 __device__ __forceinline__ float topk_softmax(float myv, int lane, int k) {
@@ -72,13 +71,20 @@ __device__ __forceinline__ void warp_argmax(float &bv, int &be) {
 // Top-k with the token's logits held in registers (E <= 32 * NPL): one read
 // of the row, then k selection rounds in registers.  Same selection rule and
 // softmax as warp_topk, hence the same result.
-template <int NPL>
+// Logit loads: from shared memory, or through L2 (.cg) so that values written
+// by other CTAs of the same kernel are seen.
+template <bool kSmem>
+__device__ __forceinline__ float load_logit(const float *row, int e) {
+  return kSmem ? row[e] : __ldcg(row + e);
+}
+
+template <int NPL, bool kSmem = false>
 __device__ __forceinline__ void warp_topk_regs(const float *row, int E, int k, int lane, int &e_out, float &w_out) {
   float v[NPL];
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
     const int e = lane + 32 * j;
-    float t = e < E ? __ldcg(row + e) : -INFINITY;
+    float t = e < E ? load_logit<kSmem>(row, e) : -INFINITY;
     if (t != t) t = -INFINITY;
     v[j] = t;
   }
@@ -164,7 +170,7 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // by counting.  Falls back to warp_topk_regs when more than 32 values pass.
 // `scratch` is 64 uint64 of shared memory private to the warp.  Same
 // selection and softmax as warp_topk, hence the same result.
-template <int NPL>
+template <int NPL, bool kSmem = false>
 __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, int lane, uint64_t *scratch,
                                                int &e_out, float &w_out) {
   uint64_t v[NPL];
@@ -172,7 +178,7 @@ __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, i
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
     const int e = lane + 32 * j;
-    v[j] = e < E ? ((uint64_t)float_key(__ldcg(row + e)) << 32) | (uint32_t)~e : 0ull;
+    v[j] = e < E ? ((uint64_t)float_key(load_logit<kSmem>(row, e)) << 32) | (uint32_t)~e : 0ull;
     m = v[j] > m ? v[j] : m;
   }
   int rank = 0;
@@ -186,7 +192,7 @@ __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, i
   const int total = __reduce_add_sync(0xffffffffu, cnt);
   if (total > 32) {
     __syncwarp();
-    warp_topk_regs<NPL>(row, E, k, lane, e_out, w_out);
+    warp_topk_regs<NPL, kSmem>(row, E, k, lane, e_out, w_out);
     return;
   }
   int base = 0;

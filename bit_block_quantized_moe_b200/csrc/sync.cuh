@@ -68,6 +68,31 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
                : "memory");
 }
 
+// ---- cp.async (load/store-unit path, 16 B per thread) ----------------------------
+// Many threads each moving 16-byte pieces keep far more bytes in flight per SM
+// than one thread issuing large bulk copies.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+// One arrival on `bar` once every cp.async this thread issued so far has landed
+// (the barrier's expected count includes it).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed cp.async groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// A warp copies `bytes` (a multiple of 16, both addresses 16-byte aligned): lane i moves pieces i, i + 32, ...
+__device__ __forceinline__ void warp_cp_async(void *dst_smem, const void *src, uint32_t bytes, int lane) {
+  uint8_t *d = static_cast<uint8_t *>(dst_smem);
+  const uint8_t *sp = static_cast<const uint8_t *>(src);
+  for (uint32_t o = (uint32_t)lane * 16u; o < bytes; o += 512u) cp_async16(d + o, sp + o);
+}
+
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
