@@ -186,7 +186,7 @@ def moe_rmsnorm_residual(resid, y, x_norm, T: int, hidden: int, eps: float = 1e-
 
 MOE_KERNEL = {"router_logits": 0, "topk": 1, "dispatch_bits": 2, "dispatch_scan": 3, "dispatch_place": 4,
               "gate_up": 5, "down": 6, "combine": 7, "decode_fused": 8,
-              "gather": 9, "frag_x": 10, "frag_h": 11}
+              "gather": 9}
 
 
 def moe_trace_kernel(kernel_id: int, before=None, after=None):

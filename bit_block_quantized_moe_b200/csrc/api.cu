@@ -52,15 +52,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_items = take((size_t)max_items * 16);
   const int max_tc_items = max_items_for(d, T, 64);
   const size_t o_tc_items = take((size_t)max_tc_items * 16);
-  const int max_g_tiles = max_items_for(d, T, 32);
-  const size_t o_g_tiles = take((size_t)max_g_tiles * 16);
-  const bool tc = T > 8 && use_tc_path(d, T);
-  const bool grouped = T > 8 && !tc;
-  const size_t o_xf = take(grouped ? (size_t)T * (H / 128) * 272 : 0);
-  const size_t o_xus = take(grouped ? (size_t)T * 4 : 0);
-  const size_t o_hf = take(grouped ? slots * (I / 128) * 272 : 0);
-  const size_t o_hus = take(grouped ? slots * 4 : 0);
-  const size_t o_xs = take(tc ? slots * H * 2 : 0);
+  const size_t o_xs = take(T > 8 ? slots * H * 2 : 0);
   const size_t o_h = take(slots * I * 2);
   const size_t o_y = take(slots * H * 4);
   const bool fused = decode_fused_supported(d, T);
@@ -86,17 +78,11 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->items = reinterpret_cast<int4 *>(b + o_items);
     ws->tc_items = reinterpret_cast<int4 *>(b + o_tc_items);
     ws->n_tc_items = reinterpret_cast<uint32_t *>(b + o_hdr + 8);
-    ws->g_tiles = reinterpret_cast<int4 *>(b + o_g_tiles);
-    ws->n_g_tiles = reinterpret_cast<uint32_t *>(b + o_hdr + 12);
-    ws->xf = b + o_xf;
-    ws->xunscale = reinterpret_cast<float *>(b + o_xus);
-    ws->hf = b + o_hf;
-    ws->hunscale = reinterpret_cast<float *>(b + o_hus);
     ws->xs = reinterpret_cast<uint16_t *>(b + o_xs);
     ws->max_tc_items = max_tc_items;
     ws->h = reinterpret_cast<uint16_t *>(b + o_h);
     ws->y = reinterpret_cast<float *>(b + o_y);
-    ws->gbar = reinterpret_cast<uint32_t *>(b + o_hdr + 64);
+    ws->gbar = reinterpret_cast<uint64_t *>(b + o_hdr + 64);
     ws->tile_cnt = reinterpret_cast<uint32_t *>(b + o_tcnt);
     ws->partial = reinterpret_cast<float *>(b + o_part);
     ws->words = (int)words;
@@ -213,14 +199,8 @@ static cudaError_t run_experts(const moe_dims &d, const uint16_t *x, const moe_e
   if (err == cudaSuccess) {
     const uint8_t *ex = static_cast<const uint8_t *>(experts->packed);
     const uint8_t *sh = static_cast<const uint8_t *>(shared->packed);
-    // few tokens: register-dequant tensor-core tiles of 8 tokens; many tokens: grouped e4m3 GEMM,
-    // or the tcgen05 GEMM once experts see enough tokens each
-    if (T <= 8)
-      err = launch_experts(d, G, ex, sh, x, T, ws, s);
-    else if (use_tc_path(d, T))
-      err = launch_tc_experts(d, G, ex, sh, x, T, ws, s);
-    else
-      err = launch_grouped_experts(d, G, ex, sh, x, T, ws, s);
+    // few tokens: register-dequant tensor-core tiles of 8 tokens; otherwise the tcgen05 grouped GEMM
+    err = T <= 8 ? launch_experts(d, G, ex, sh, x, T, ws, s) : launch_tc_experts(d, G, ex, sh, x, T, ws, s);
   }
   if (err == cudaSuccess) err = launch_combine(d, T, ws, out, s);
   return err;

@@ -62,7 +62,7 @@ struct DecodeArgs {
   uint16_t *h;         // [T][k+1][I]
   float *partial;      // [entries][dn_units][32][4]
   uint32_t *tile_cnt;  // [dn_units] then ready[kMaxEntries]
-  uint32_t *gbar;      // [0] count, [1] generation
+  uint64_t *gbar;      // monotonic grid-barrier arrival counter
   int32_t *idx_out;    // optional [T][k]
   float *w_out;        // optional [T][k]
   uint16_t *out;       // [T][H]
@@ -199,16 +199,13 @@ __device__ void build_b_fragments(const uint16_t *v, int stride, int K, int T, i
 // 4 * quad + c, in units of 2^(s_t - 9).  Four block tiles per group are
 // staged: loads, code masking, one m16n8k32 MMA per quad (accumulator started
 // at the block's correction), then the fp16 block scales.
+// Block groups [grp0, grp1) of a unit whose K spans n_groups groups; adds to acc.
 template <int NQ>
-__device__ __forceinline__ void unit_gemv(const uint8_t *st, int n_groups, const uint2 *frag, const float *corr,
-                                          int lane, float (&acc)[2][4]) {
+__device__ __forceinline__ void unit_gemv(const uint8_t *st, int grp0, int grp1, int n_groups, const uint2 *frag,
+                                          const float *corr, int lane, float (&acc)[2][4]) {
   const int g = lane >> 2, c = lane & 3;
   const int nb = n_groups * 4;
-#pragma unroll
-  for (int qd = 0; qd < 2; ++qd)
-#pragma unroll
-    for (int r = 0; r < 4; ++r) acc[qd][r] = 0.f;
-  for (int grp = 0; grp < n_groups; ++grp) {
+  for (int grp = grp0; grp < grp1; ++grp) {
     const uint8_t *gp = st + (size_t)grp * kGroupBytes;
     const uint4 cw = lds128(gp + lane * 16);
     const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
@@ -334,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       }
       named_bar(kBarConsumers, kConsumers);
     }
-    grid_barrier(&a.gbar[0], &a.gbar[1], kBarConsumers, kConsumers, tid == 0, a.status, &misc[2]);
+    grid_barrier(a.gbar, kBarConsumers, kConsumers, tid == 0, a.status, &misc[2]);
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
     // All logits into shared memory first (one coalesced pass through L2), then one warp per token.
@@ -412,55 +409,72 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const int g1 = (int)((long long)n_gu * (blockIdx.x + 1) / gridDim.x);
   const int d0 = (int)((long long)n_dn * blockIdx.x / gridDim.x);
   const int d1 = (int)((long long)n_dn * (blockIdx.x + 1) / gridDim.x);
-  const int pps = (int)(a.stage_bytes / G.dn_unit_bytes);  // down pairs per stage
+  const int pps = 2;  // down units (16 rows) per stage: enough stages to keep every warp busy
   const int n_gu_st = g1 - g0;
   const int n_dn_st = (d1 - d0 + pps - 1) / pps;
   const int n_st = n_gu_st + n_dn_st;
-  // Stage s belongs to warp s % nw, which copies it (cp.async) into one of its
-  // own spw ring slots, waits for its own copies, computes it and refills the
-  // slot with its stage s + spw * nw.  No other warp touches the slot.
-  const int nw = a.nw, spw = a.ns / a.nw;
+  // Stage s belongs to warp s % nw, which copies it (cp.async) into its own
+  // ring slot, waits for its own copies, computes it and refills the slot with
+  // its next stage s + nw.  No other warp touches the slot.
+  const int nw = a.nw, spw = 1;
   auto expert_ptr = [&](int entry) -> const uint8_t * {
     const int e = ent[entry];
     return e == E ? a.shared : a.experts + (size_t)e * G.expert_bytes;
   };
   auto stage_ptr = [&](int s) { return ring + (size_t)(warp * spw + (s / nw) % spw) * a.stage_bytes; };
-  auto issue_stage = [&](int s) {  // one commit group per call, empty past the last stage
-    if (s < n_st) {
-      uint8_t *dst = stage_ptr(s);
-      if (s < n_gu_st) {
-        const int id = g0 + s;
-        warp_cp_async(dst, expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes,
-                      (uint32_t)G.gu_unit_bytes, lane);
-      } else {
-        const int q0 = d0 + (s - n_gu_st) * pps, q1 = min(d1, q0 + pps);
-        for (int q = q0; q < q1; ++q)
-          warp_cp_async(dst + (size_t)(q - q0) * G.dn_unit_bytes,
-                        expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes,
-                        (uint32_t)G.dn_unit_bytes, lane);
+  // A stage is copied as 4 commit groups (its quarters, in order) so that the
+  // warp can start on the first quarter while the rest is still arriving:
+  // gate/up = one unit (quarter = 4 block groups), down = 2 units of 16 rows
+  // (quarter = half a unit).  Past the last stage the groups are empty.
+  auto issue_stage = [&](int s) {
+    for (int qt = 0; qt < 4; ++qt) {
+      if (s < n_st) {
+        uint8_t *dst = stage_ptr(s);
+        if (s < n_gu_st) {
+          const int id = g0 + s;
+          const size_t qb = G.gu_unit_bytes / 4;
+          warp_cp_async(dst + qt * qb,
+                        expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes + qt * qb,
+                        (uint32_t)qb, lane);
+        } else {
+          const int q = d0 + (s - n_gu_st) * pps + (qt >> 1);
+          const size_t hb2 = G.dn_unit_bytes / 2;
+          if (q < d1)
+            warp_cp_async(dst + (size_t)(qt >> 1) * G.dn_unit_bytes + (qt & 1) * hb2,
+                          expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes +
+                              (qt & 1) * hb2,
+                          (uint32_t)hb2, lane);
+        }
       }
+      cp_async_commit();
     }
-    cp_async_commit();
   };
-  auto wait_stage = [&]() {  // the oldest of this warp's spw outstanding stages has landed
-    if (spw == 1)
-      cp_async_wait_group<0>();
-    else
+  // quarter qt of the warp's current stage has landed (spw == 1: nothing newer is in flight)
+  auto wait_quarter = [&](int qt) {
+    if (qt == 0)
+      cp_async_wait_group<3>();
+    else if (qt == 1)
+      cp_async_wait_group<2>();
+    else if (qt == 2)
       cp_async_wait_group<1>();
+    else
+      cp_async_wait_group<0>();
     __syncwarp();
   };
-  if (warp < nw)
-    for (int j = 0; j < spw; ++j) issue_stage(warp + j * nw);
+  if (warp < nw) issue_stage(warp);
 
   // ---------------- consumers, phase C: gate/up + SwiGLU ----------------
   for (int s_idx = warp; warp < nw && s_idx < n_gu_st; s_idx += nw) {
-    wait_stage();
     const uint8_t *st = stage_ptr(s_idx);
-    float acc[2][4];
-    if (nq == 1)
-      unit_gemv<1>(st, G.gu_groups, xb, corr, lane, acc);
-    else
-      unit_gemv<2>(st, G.gu_groups, xb, corr, lane, acc);
+    float acc[2][4] = {};
+    const int gq = G.gu_groups / 4;  // block groups per quarter
+    for (int qt = 0; qt < 4; ++qt) {
+      wait_quarter(qt);
+      if (nq == 1)
+        unit_gemv<1>(st, qt * gq, (qt + 1) * gq, G.gu_groups, xb, corr, lane, acc);
+      else
+        unit_gemv<2>(st, qt * gq, (qt + 1) * gq, G.gu_groups, xb, corr, lane, acc);
+    }
     __syncwarp();
     issue_stage(s_idx + spw * nw);
     const int id = g0 + s_idx;
@@ -519,7 +533,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
 
   for (int s_idx = n_gu_st + ((warp - n_gu_st % nw + nw) % nw); warp < nw && s_idx < n_st; s_idx += nw) {
     const int sd = s_idx - n_gu_st;
-    wait_stage();
     const uint8_t *st = stage_ptr(s_idx);
     const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
     for (int q = q0; q < q1; ++q) {
@@ -527,11 +540,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       const uint8_t *pp_st = st + (size_t)(q - q0) * G.dn_unit_bytes;
       const uint2 *hbe = hb + he * nq * (kMaxI / 32) * 32;
       const float *hce = hcorr + he * (kMaxI / 32) * kMaxTok;
-      float acc[2][4];
-      if (nq == 1)
-        unit_gemv<1>(pp_st, G.dn_groups, hbe, hce, lane, acc);
-      else
-        unit_gemv<2>(pp_st, G.dn_groups, hbe, hce, lane, acc);
+      float acc[2][4] = {};
+      const int hg = G.dn_groups / 2;  // block groups per half unit
+      for (int h2 = 0; h2 < 2; ++h2) {
+        wait_quarter(2 * (q - q0) + h2);
+        if (nq == 1)
+          unit_gemv<1>(pp_st, h2 * hg, (h2 + 1) * hg, G.dn_groups, hbe, hce, lane, acc);
+        else
+          unit_gemv<2>(pp_st, h2 * hg, (h2 + 1) * hg, G.dn_groups, hbe, hce, lane, acc);
+      }
       // partial tile layout: lane (g, c) -> {row g tok c, row g+8 tok c, row g tok c+4, row g+8 tok c+4}
       float o4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -606,6 +623,7 @@ bool decode_fused_supported(const moe_dims &d, int T) {
   const PackedGeom G = packed_geom(d.hidden, d.inter);
   if (T < 1 || T > kMaxTok || T * d.top_k > kMaxSel || d.n_experts > kMaxE) return false;
   if (G.dn_groups != 4) return false;  // down: 4 groups of 128 (inter 512, the h cache size)
+  if (G.gu_groups % 4) return false;   // gate/up units stream in quarters of whole block groups
   return true;
 }
 
@@ -630,8 +648,8 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   const SmemLayout L0 = smem_layout(T, G.H, 0, stage_bytes);
   const int slots = (int)((max_smem - (int)L0.ring - 128) / (int)stage_bytes);
   if (slots < 1) return cudaErrorInvalidConfiguration;
-  const int nw = min(kConsumerWarps, slots);        // warps streaming and computing stages
-  const int ns = nw * min(2, slots / nw);           // 1 or 2 private slots per warp
+  const int nw = min(kConsumerWarps, slots);  // warps streaming and computing stages, one slot each
+  const int ns = nw;
   const SmemLayout L = smem_layout(T, G.H, ns, stage_bytes);
   if (L.total > (uint32_t)max_smem) return cudaErrorInvalidConfiguration;
   // the per-CTA down range must fit the 128-entry completed-tile list

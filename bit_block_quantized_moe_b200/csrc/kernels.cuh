@@ -25,16 +25,10 @@ struct Workspace {
   int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)
   int4 *tc_items;          // [max_tc_items]: (expert, first position, tokens <= 64, 0)
   uint32_t *n_tc_items;
-  int4 *g_tiles;           // [max_g_tiles]: (expert, first position, tokens <= 32, 0)
-  uint32_t *n_g_tiles;
-  uint8_t *xf;             // [T][H/128][272 B]: e4m3 B records + block corrections of the tokens (grouped path)
-  float *xunscale;         // [T]
-  uint8_t *hf;             // [T*k + T][I/128][272 B]: the same for h
-  float *hunscale;         // [T*k + T]
-  uint16_t *xs;            // [T*k + T][H] bf16 token rows in sorted-position order (tcgen05 path)
+  uint16_t *xs;            // [T*k + T][H] bf16 token rows in sorted-position order
   uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position
   float *y;                // [T*k + T][H] fp32 expert outputs by sorted position
-  uint32_t *gbar;          // grid barrier of the fused decode kernel: count, generation (kept zeroed)
+  uint64_t *gbar;          // grid barrier of the fused decode kernel: monotonic arrival counter
   uint32_t *tile_cnt;      // fused decode: per-tile arrival counters, then per-expert ready counters
   float *partial;          // fused decode: per (expert, tile) partial outputs
   int words;               // ceil(T / 32)
@@ -57,10 +51,6 @@ cudaError_t launch_experts(const moe_dims &d, const PackedGeom &G, const uint8_t
                            const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                               const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
-cudaError_t launch_grouped_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts,
-                                   const uint8_t *shared, const uint16_t *x, int T, const Workspace &ws,
-                                   cudaStream_t s);
-bool use_tc_path(const moe_dims &d, int T);
 cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s);
 bool decode_fused_supported(const moe_dims &d, int T);
 size_t decode_partial_floats(const moe_dims &d, int T);

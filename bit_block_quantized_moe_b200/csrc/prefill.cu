@@ -333,14 +333,6 @@ bool make_maps(TcMaps *m, const uint8_t *experts, const uint8_t *shared, const P
 
 }  // namespace
 
-// The tcgen05 GEMM takes over from the grouped e4m3 path once the routed
-// experts average this many tokens each.
-constexpr long long kTcMinTokensPerExpert = 1LL << 40;
-
-bool use_tc_path(const moe_dims &d, int T) {
-  return (long long)T * d.top_k >= kTcMinTokensPerExpert * d.n_experts;
-}
-
 size_t tc_smem_bytes() { return (size_t)kStages * kStageBytes + sizeof(Bars) + 1024; }
 
 cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,

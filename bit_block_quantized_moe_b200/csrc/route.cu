@@ -321,7 +321,6 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
                                                             int T, int k, uint32_t *__restrict__ wprefix,
                                                             int32_t *counts, int32_t *offsets, int4 *items,
                                                             uint32_t *n_items, int4 *tc_items, uint32_t *n_tc_items,
-                                                            int4 *g_tiles, uint32_t *n_g_tiles,
                                                             uint32_t *done_counter) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -351,36 +350,31 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
   if (!is_last) return;
   __threadfence();
   // Work items: (expert, first sorted position, tokens) in tiles of 8 tokens
-  // (register-dequant path), 32 tokens (grouped e4m3 path) and 64 tokens
-  // (tcgen05 path).
-  __shared__ int s_cnt[256], s_items[256], s_tc[256], s_g[256];
+  // (register-dequant path) and of 64 tokens (tcgen05 path).
+  __shared__ int s_cnt[256], s_items[256], s_tc[256];
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int eb = threadIdx.x * per, ee = min(E, eb + per);
-  int my_cnt = 0, my_items = 0, my_tc = 0, my_g = 0;
+  int my_cnt = 0, my_items = 0, my_tc = 0;
   for (int i = eb; i < ee; ++i) {
     const int c = ((volatile int32_t *)counts)[i];
     my_cnt += c;
     my_items += (c + 7) >> 3;
     my_tc += (c + 63) >> 6;
-    my_g += (c + 31) >> 5;
   }
   s_cnt[threadIdx.x] = my_cnt;
   s_items[threadIdx.x] = my_items;
   s_tc[threadIdx.x] = my_tc;
-  s_g[threadIdx.x] = my_g;
   __syncthreads();
   if (threadIdx.x == 0) {  // tiny serial scan over 256 partial sums
-    int a = 0, b = 0, tc = 0, gt = 0;
+    int a = 0, b = 0, tc = 0;
     for (int i = 0; i < (int)blockDim.x; ++i) {
-      const int ca = s_cnt[i], cb = s_items[i], cc = s_tc[i], cg = s_g[i];
+      const int ca = s_cnt[i], cb = s_items[i], cc = s_tc[i];
       s_cnt[i] = a;
       s_items[i] = b;
       s_tc[i] = tc;
-      s_g[i] = gt;
       a += ca;
       b += cb;
       tc += cc;
-      gt += cg;
     }
     offsets[E] = a;  // == T * k
     const int shared_items = (T + 7) >> 3;
@@ -389,18 +383,14 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
     const int shared_tc = (T + 63) >> 6;
     for (int i = 0; i < shared_tc; ++i) tc_items[tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
     *n_tc_items = (uint32_t)(tc + shared_tc);
-    const int shared_g = (T + 31) >> 5;
-    for (int i = 0; i < shared_g; ++i) g_tiles[gt + i] = make_int4(E, T * k + 32 * i, min(32, T - 32 * i), 0);
-    *n_g_tiles = (uint32_t)(gt + shared_g);
   }
   __syncthreads();
-  int pos = s_cnt[threadIdx.x], it = s_items[threadIdx.x], itc = s_tc[threadIdx.x], ig = s_g[threadIdx.x];
+  int pos = s_cnt[threadIdx.x], it = s_items[threadIdx.x], itc = s_tc[threadIdx.x];
   for (int i = eb; i < ee; ++i) {
     const int c = ((volatile int32_t *)counts)[i];
     offsets[i] = pos;
     for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
     for (int j = 0; j < c; j += 64) tc_items[itc++] = make_int4(i, pos + j, min(64, c - j), 0);
-    for (int j = 0; j < c; j += 32) g_tiles[ig++] = make_int4(i, pos + j, min(32, c - j), 0);
     pos += c;
   }
 }
@@ -461,8 +451,8 @@ cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaS
   const int E = d.n_experts, k = d.top_k;
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, false, s);
   dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, s>>>(ws.bitmap, ws.words, E, T, k, ws.wprefix, ws.counts, ws.offsets,
-                                                   ws.items, ws.n_items, ws.tc_items, ws.n_tc_items, ws.g_tiles,
-                                                   ws.n_g_tiles, ws.done_counter);
+                                                   ws.items, ws.n_items, ws.tc_items, ws.n_tc_items,
+                                                   ws.done_counter);
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, true, s);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;

@@ -119,34 +119,34 @@ __device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
 __device__ __forceinline__ uint2 ldg_cg_v2(const void *p) { return __ldcg(reinterpret_cast<const uint2 *>(p)); }
 __device__ __forceinline__ float4 ldg_cg_f4(const void *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
 
-// Grid-wide barrier for a co-resident (cooperatively launched) grid.  The
-// participating threads of each CTA first meet at named barrier `bar_id`;
-// thread `leader` arrives on the global counter; the last CTA to arrive resets
-// the counter and bumps the generation word the others wait on.  Leaves
-// count == 0, so the next barrier (or the next launch) starts clean.
-// Returns false (and sets the status timeout bit) if the wait hit the limit.
-__device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t *gen, int bar_id, int nthreads, bool leader,
-                                             uint32_t *status, int *flag_smem) {
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier for a co-resident (cooperatively launched) grid, over one
+// monotonic 64-bit arrival counter (zeroed once with the workspace, never
+// reset).  The participating threads of each CTA meet at named barrier
+// `bar_id`; thread `leader` fences, adds 1 and waits until the counter reaches
+// the next multiple of gridDim.x: one atomic round trip per CTA.  Returns false
+// (and sets the status timeout bit) if the wait hit the limit.
+__device__ __forceinline__ bool grid_barrier(uint64_t *count, int bar_id, int nthreads, bool leader, uint32_t *status,
+                                             int *flag_smem) {
   named_bar(bar_id, nthreads);
   if (leader) {
     bool ok = true;
-    const uint32_t g = ld_acquire_gpu(gen);
     __threadfence();
-    const uint32_t arrived = atomicAdd(count, 1u) + 1u;
-    if (arrived == gridDim.x) {
-      atomicExch(count, 0u);
-      __threadfence();
-      st_release_gpu(gen, g + 1u);
-    } else {
-      const uint64_t t0 = global_timer_ns();
-      while (ld_acquire_gpu(gen) == g) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-          set_status(status, kStatusTimeout);
-          ok = false;
-          break;
-        }
-        __nanosleep(32);
+    const unsigned long long old = atomicAdd(reinterpret_cast<unsigned long long *>(count), 1ull);
+    const uint64_t target = (old / gridDim.x + 1) * gridDim.x;
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu_u64(count) < target) {
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        set_status(status, kStatusTimeout);
+        ok = false;
+        break;
       }
+      __nanosleep(32);
     }
     *flag_smem = ok ? 0 : 1;
   }

@@ -107,9 +107,11 @@ moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_ex
 /* ---- workspace --------------------------------------------------------------
  * Host.  Bytes of scratch memory moe_route / moe_layer_forward /
  * moe_experts_forward need for up to max_T tokens (0 if invalid).  Its first
- * 4 bytes hold the sticky device status word: zero the workspace (or at least
- * those 4 bytes) once after allocating it.  One workspace must not be used by
- * two calls that can run at the same time. */
+ * 256 bytes hold the sticky device status word (offset 0) and the decode
+ * kernel's grid-barrier counter (offset 64): zero the workspace (or at least
+ * those 256 bytes) once after allocating it, and again after a call reported
+ * MOE_ERR_TIMEOUT.  One workspace must not be used by two calls that can run
+ * at the same time. */
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T);
 
 /* ---- routing ------------------------------------------------------------------
@@ -197,9 +199,7 @@ enum {
   MOE_KERNEL_DOWN = 6,
   MOE_KERNEL_COMBINE = 7,
   MOE_KERNEL_DECODE_FUSED = 8,
-  MOE_KERNEL_GATHER = 9,
-  MOE_KERNEL_FRAG_X = 10,
-  MOE_KERNEL_FRAG_H = 11
+  MOE_KERNEL_GATHER = 9
 };
 moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after);
 

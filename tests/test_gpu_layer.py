@@ -7,6 +7,10 @@ import oracle
 from gen import CONFIGS, MoeConfig, make_x
 from parity import GAP_TIE, W_TOL, build_layer, check_layer, check_routing, gpu_forward, to_dev_bf16
 
+
+def bf16_to_f32(bits):
+    return (np.asarray(bits).view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+
 pytestmark = pytest.mark.gpu
 
 
@@ -197,3 +201,59 @@ def test_fused_decode_agrees_with_route_and_general_path(full):
     torch.cuda.synchronize()
     yg = (out.cpu().numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
     assert np.max(np.abs(yg - y1)) <= 4e-3 * np.max(np.abs(y1))
+
+
+def test_config3_stack_layer_by_layer():
+    """48-layer stack (config 3), checked on its first 3 seeded layers: x_0 = x; layer l
+    reads bf16(RMSNorm(resid_l)); resid_{l+1} = resid_l + y_l (fp32 on the GPU).  Each
+    step is compared on 256 sampled tokens: the GPU's RMSNorm output against the
+    oracle's RMSNorm of the GPU residual, and the GPU layer against the oracle layer on
+    the GPU's own bf16 layer input.  Every layer applies the same code to its own
+    weights, so the first layers stand for the rest; the full 24 GB stack is the
+    bench's workload."""
+    from bit_block_quantized_moe_b200 import moe_rmsnorm_residual
+
+    cfg = CONFIGS[3]
+    T, H = cfg.tokens, cfg.hidden
+    rng = np.random.default_rng(3)
+    sample = np.sort(rng.choice(T, 256, replace=False))
+    x0 = make_x(cfg, seed=0)
+    resid = torch.from_numpy(bf16_to_f32(x0)).cuda()
+    xn = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6)
+    for layer in range(3):
+        torch.cuda.synchronize()
+        r_host = resid.cpu().numpy().astype(np.float64)
+        xn_host = xn.cpu().numpy().view(np.uint16)
+        want = oracle.rmsnorm(r_host[sample], 1e-6)
+        got = bf16_to_f32(xn_host[sample])
+        assert np.max(np.abs(got - want) / np.maximum(np.abs(want), 1e-3)) < 2 ** -8
+        L, w = build_layer(cfg, layer=layer)
+        idx = torch.full((T, cfg.top_k), -1, dtype=torch.int32, device="cuda")
+        wts = torch.zeros((T, cfg.top_k), dtype=torch.float32, device="cuda")
+        y = L.forward(xn, topk_idx=idx, topk_w=wts)
+        torch.cuda.synchronize()
+        L.check_status()
+        err, l2, flagged = check_layer(cfg, w, xn_host, bf16_to_f32(y.cpu().numpy().view(np.uint16)).astype(np.float64),
+                                       idx.cpu().numpy(), wts.cpu().numpy(), tokens=sample)
+        print(f"stack layer {layer}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+        moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6)  # resid += y; next layer input
+        del L
+
+
+def test_config4_prefill_32k(full):
+    """Config 4: a T = 32768 prefill chunk through a full-size Zipf layer: routing of
+    every token against the oracle, outputs on 256 sampled tokens (plus the flagged
+    ones and both ends).  The decode sweep T in {1, 2, 3} on the same weights is
+    test_decode_window_full_size."""
+    cfg = CONFIGS[4]
+    L, w = full
+    x = make_x(cfg, seed=4)
+    y, idx, wts = gpu_forward(L, x)
+    idx_o, w_o, gap, _ = oracle.route(x, w["router_w"], w["router_b"], cfg.top_k)
+    flagged = check_routing(idx, wts, idx_o, w_o, gap)
+    rng = np.random.default_rng(4)
+    sample = np.union1d(rng.choice(cfg.tokens, 256, replace=False), np.array(flagged, dtype=np.int64))
+    sample = np.union1d(sample, [0, cfg.tokens - 1])
+    err, l2, _ = check_layer(cfg, w, x, y, idx, wts, tokens=sample)
+    print(f"config4 T=32768: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
