@@ -125,51 +125,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
 }
 
-// ---- e4m3 path (few-token GEMV on m16n8k32 fp8 MMAs) ------------------------------
-// The same code word also feeds an m16n8k32 e4m3 MMA with no arithmetic: a
-// byte v < 16 is the e4m3 value v * 2^-9 (subnormal for v < 8, exponent 1
-// above, one contiguous scale), so masking the codes of one row into bytes
-// gives q * 2^-9 (mask 0x03 per byte) or 4q * 2^-9 (mask 0x0C; the B operand
-// of those k carries 1/4).  Register m of the A fragment (rows g, g+8; k'
-// 4c..4c+3, 16+4c..16+4c+3) holds, byte i, the code of block position
-//   a0 / a1 (rows g / g+8):  4c + {0, 16, 1, 17}[i]
-//   a2 / a3 (rows g / g+8):  4c + {2, 18, 3, 19}[i]   (value 4q)
-// The B fragment must list the activations in the same order.
-__device__ __forceinline__ void decode_q2_e4m3(uint32_t w, uint32_t (&a)[4]) {
-  const uint32_t w4 = w >> 4;
-  a[0] = w & 0x03030303u;
-  a[1] = w4 & 0x03030303u;
-  a[2] = w & 0x0C0C0C0Cu;
-  a[3] = w4 & 0x0C0C0C0Cu;
-}
-// Block position of byte i of A register 0/1 (k_lo) and 2/3 (k_hi) for lane column c.
-__host__ __device__ constexpr int e4m3_k_lo(int c, int i) { return 4 * c + (i & 1) * 16 + (i >> 1); }
-__host__ __device__ constexpr int e4m3_k_hi(int c, int i) { return 4 * c + 2 + (i & 1) * 16 + (i >> 1); }
-
-// Two-term e4m3 split of a bf16 value v already scaled into [2^-2, 256): the
-// high term keeps sign, exponent and the top 3 mantissa bits, the low term is
-// the remaining 4 bits; both are e4m3 values and hi + lo == v exactly.
-// Smaller magnitudes lose the bits below 2^-9 (absolute error <= 2^-10).
-__device__ __forceinline__ float e4m3_split_hi(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFF00000u); }
-
-// Four floats to four e4m3 bytes (value 0 in byte 0), round to nearest, saturating.
-__device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
-  uint16_t lo, hi;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(v1), "f"(v0));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(v3), "f"(v2));
-  return (uint32_t)lo | ((uint32_t)hi << 16);
-}
-
-// D = A(16x32 e4m3) * B(32x8 e4m3) + C, fp32 accumulate.
-__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
-                                               const float (&c)[4]) {
-  asm(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%10,%11,%12,%13};\n"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
-}
-
 // (a0, a1) += (s, s) * (d0, d1): one packed fp32x2 FMA (sm_100), each lane rounded like fmaf.
 __device__ __forceinline__ void fma2_bcast(float &a0, float &a1, float s, float d0, float d1) {
   uint64_t acc, dd, ss;
@@ -179,15 +134,6 @@ __device__ __forceinline__ void fma2_bcast(float &a0, float &a1, float s, float 
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(ss), "l"(dd));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
 }
-
-// Power-of-two scale exponent s for a vector with max |v| = m: m * 2^s in [128, 256)
-// (s = 0 for m == 0), clamped to [-100, 120] so that 2^s and 2^(9-s) stay normal fp32 values.
-__device__ __forceinline__ int e4m3_scale_exp(float m) {
-  if (!(m > 0.f)) return 0;
-  const int e = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;  // m is normal for bf16 inputs >= 2^-126
-  return max(-100, min(120, 7 - e));
-}
-__device__ __forceinline__ float exp2_int(int s) { return __uint_as_float((uint32_t)(127 + s) << 23); }
 
 // Read-only global load through the non-coherent path (weights, router).
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }

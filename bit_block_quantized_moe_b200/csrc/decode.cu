@@ -6,7 +6,8 @@
 //     CTA's router rows into shared memory and prefetches its slice of the
 //     shared expert into L2.  Consumers compute the router rows (2 warps per row, one
 //     half of K each) and the correction sums of the biased decode.
-//     -- grid barrier: all logits written --
+//     -- grid barrier: all logits written (the token fragments are built
+//        between arriving and waiting) --
 //  B  Every CTA selects the top-k of every token (threshold + rank, one warp
 //     per token) and builds the same sorted list of touched experts plus the
 //     shared expert.
@@ -24,14 +25,13 @@
 //     partial = w[t, e] * (Wd_e h_e) per (expert, tile).  The last CTA to
 //     contribute to a tile sums its partials in expert order and writes out
 //     (bf16).
-// Weights reach the tensor cores with no arithmetic: the 2-bit codes of a
-// row are masked into e4m3 bytes (value q * 2^-9) that form the A fragment of
-// an m16n8k32 fp8 MMA.  The tokens form the B fragment: each token vector is
-// scaled by a power of two and split into two e4m3 terms (columns 2t and
-// 2t+1, 4 tokens per MMA), exact for every element above 2^-8 of the
-// vector's largest.  The -1 of d * (q - 1) starts the accumulator at minus the
-// block sum of the token, and the fp16 block scale d multiplies each block's
-// fp32 result.  Every wait is bounded (sync.cuh).
+// Dequantisation happens in registers: the 2-bit codes of a row OR into the
+// mantissa of bf16 128.0 (128 + q, or 128 + 4q with the matching activation
+// pair pre-scaled by 1/4), one logic op per pair of weights, and feed
+// m16n8k16 tensor-core MMAs with the tokens as the 8 columns.  The -1 of
+// d * (q - 1) and the 128 bias start the accumulator at minus the weighted
+// block sum of the token; the fp16 block scale d multiplies each block's fp32
+// result.  All products are exact.  Every wait is bounded (sync.cuh).
 #include "kernels.cuh"
 #include "router.cuh"
 #include "sync.cuh"
@@ -73,35 +73,23 @@ struct DecodeArgs {
 };
 
 struct SmemLayout {
-  uint32_t xs, corr, xb, xsc, hb, hcorr, hsc, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc,
-      ring, total;
+  uint32_t xs, corr, hcorr, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc, ring, total;
 };
-
-// Token quads: the 8 columns of an m16n8k32 MMA hold 4 tokens x 2 split terms.
-__host__ __device__ inline int token_quads(int T) { return (T + 3) / 4; }
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes) {
   SmemLayout L;
   uint32_t o = 0;
-  // xs: the tokens (bf16 rows, phase A).  The same bytes hold the h fragments of phase D.
-  const uint32_t hb_bytes = 2u * token_quads(T) * (kMaxI / 32) * 256;
-  const uint32_t hcorr_bytes = 2u * (kMaxI / 32) * kMaxTok * 4;
-  const uint32_t xs_bytes = (uint32_t)T * (H + 16) * 2;
-  L.xs = o;
-  L.hb = o;  // [2 cached experts][quads][I/32][32] B fragments of h
-  L.hcorr = o + hb_bytes;  // [2][I/32][8]
-  L.hsc = L.hcorr + hcorr_bytes;  // [2][8]
-  o = align_to(o + max(xs_bytes, hb_bytes + hcorr_bytes + 2u * kMaxTok * 4), 16);
-  L.corr = o;  // [H/32 blocks][8 tokens]: -2^-9 * sum of the scaled tokens over the block
+  L.xs = o;  // [T + 1][H + 16] bf16 token rows (the B operand once prepared); row T stays zero
+  o = align_to(o + (uint32_t)(T + 1) * (H + 16) * 2, 16);
+  L.corr = o;  // [H/32 blocks][8 tokens] accumulator starts of the biased decode
   o = align_to(o + (uint32_t)(H / 32) * kMaxTok * 4, 16);
-  L.xb = o;  // [quads][H/32 blocks][32 lanes] B fragments (uint2) of the scaled, split tokens
-  o = align_to(o + (uint32_t)token_quads(T) * (H / 32) * 256, 16);
-  L.xsc = o;  // [8] 2^(9 - s_t): undoes the token scale and the 2^-9 of the A bytes
-  o += kMaxTok * 4;
+  L.hcorr = o;  // [2 cached experts][I/32][8]
+  o = align_to(o + 2u * (kMaxI / 32) * kMaxTok * 4, 16);
   L.rpart = o;  // [rows per pass][8 tokens][router parts]
   o += (kConsumerWarps / kRouterParts) * kMaxTok * kRouterParts * 4;
+  o = align_to(o, 16);
   L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
   o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
   L.sel_idx = o;
@@ -118,129 +106,84 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   o = align_to(o + kMaxEntries * kMaxTok, 16);
   L.tokw = o;
   o = align_to(o + kMaxEntries * kMaxTok * 4, 16);
-  L.misc = o;  // [0] entries [1] abort [2] barrier flag [3] done tiles [8..15] token scale exponents
+  L.misc = o;  // [0] entries [1] abort [2] barrier flag [3] done tiles
   o += 64;
   L.ring = align_to(o, 128);
   L.total = L.ring + (uint32_t)ns * stage_bytes;
   return L;
 }
 
-// Per-token power-of-two scales, block correction sums and e4m3 B fragments of
-// the vectors v[t][0..K) (bf16 rows `stride` elements apart), t < T.  All
-// consumer threads call it (it holds named barriers).
-//   unscale[t] = 2^(9 - s_t), with max_k |v[t][k]| * 2^s_t in [128, 256);
-//   corr[b][t] = -2^-9 * sum_{k in block b} v[t][k] * 2^s_t  (the -1 of q - 1);
-//   frag[(quad * nb + b) * 32 + lane]: lane (g, c) holds column g = 2 * (t % 4)
-//   + split term, rows k in block order e4m3_k_lo (x) / e4m3_k_hi (x, times 1/4).
-__device__ void build_b_fragments(const uint16_t *v, int stride, int K, int T, int nq, uint2 *frag, float *corr,
-                                  float *unscale, int *sexp, int warp, int lane, int tid) {
-  const int nb = K / 32;
-  if (warp < T) {
-    uint32_t m = 0;  // largest |v| as a bf16 bit pattern (ordered like the magnitudes)
-    for (int i = lane; i < K / 8; i += 32) {
-      const uint4 u = *reinterpret_cast<const uint4 *>(v + warp * stride + 8 * i);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// Prepares T bf16 rows v[t][0..K) (`stride` elements apart, t < T) in shared
+// memory as the B operand of the biased decode (decode_q2_biased): for every
+// 32-wide block b, corr[b][t] = -(129 * sum_{k%4<2} v[t][k] + 33 * sum_{k%4>=2}
+// v[t][k]), then the pairs (4c+2, 4c+3) of every four are scaled by 1/4 in place
+// (exact).  The MMA of codes 128 + q / 128 + 4q against these rows, started at
+// corr, gives sum_k (q_k - 1) v[t][k].  One thread per (block, token).
+__device__ __forceinline__ void prep_rows(uint16_t *v, int stride, int K, int T, float *corr, int tid) {
+  for (int i = tid; i < (K / 32) * T; i += kConsumers) {
+    const int b = i / T, t = i % T;
+    uint4 *xr = reinterpret_cast<uint4 *>(v + t * stride + 32 * b);
+    float s129 = 0.f, s33 = 0.f;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) m = max(m, max(w[h] & 0x7FFFu, (w[h] >> 16) & 0x7FFFu));
+    for (int q = 0; q < 4; ++q) {
+      uint4 w = xr[q];
+      s129 += __uint_as_float(w.x << 16) + __uint_as_float(w.x & 0xffff0000u);
+      s33 += __uint_as_float(w.y << 16) + __uint_as_float(w.y & 0xffff0000u);
+      s129 += __uint_as_float(w.z << 16) + __uint_as_float(w.z & 0xffff0000u);
+      s33 += __uint_as_float(w.w << 16) + __uint_as_float(w.w & 0xffff0000u);
+      w.y = bf16x2_fma(w.y, 0x3E803E80u, 0x80008000u);
+      w.w = bf16x2_fma(w.w, 0x3E803E80u, 0x80008000u);
+      xr[q] = w;
     }
-    m = __reduce_max_sync(0xffffffffu, m);
-    if (lane == 0) {
-      const int sx = e4m3_scale_exp(__uint_as_float(m << 16));
-      sexp[warp] = sx;
-      unscale[warp] = 512.f * exp2_int(-sx);
-    }
+    corr[b * kMaxTok + t] = -(129.f * s129 + 33.f * s33);
   }
-  named_bar(kBarConsumers, kConsumers);
-  for (int i = tid; i < nb * kMaxTok; i += kConsumers) {
-    const int b = i / kMaxTok, t = i % kMaxTok;
-    float sum = 0.f;
-    if (t < T) {
-      const float sc = exp2_int(sexp[t]);
-      const uint4 *row = reinterpret_cast<const uint4 *>(v + t * stride + 32 * b);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 u = row[q];
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          sum = fmaf(__uint_as_float(w[h] << 16), sc, sum);
-          sum = fmaf(__uint_as_float(w[h] & 0xffff0000u), sc, sum);
-        }
-      }
-    }
-    corr[b * kMaxTok + t] = -sum * (1.f / 512.f);
-  }
-  for (int i = tid; i < nq * nb * 32; i += kConsumers) {
-    const int qd = i / (nb * 32), r = i % (nb * 32), b = r / 32, ln = r % 32;
-    const int gq = ln >> 2, cq = ln & 3, t = 4 * qd + (gq >> 1), part = gq & 1;
-    uint2 f = make_uint2(0u, 0u);
-    if (t < T) {
-      const float sc = exp2_int(sexp[t]);
-      const uint16_t *row = v + t * stride + 32 * b;
-      float lo[4], hi[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float vl = bf16_bits_to_float(row[e4m3_k_lo(cq, j)]) * sc;
-        const float vh = bf16_bits_to_float(row[e4m3_k_hi(cq, j)]) * sc * 0.25f;
-        const float hl = e4m3_split_hi(vl), hh = e4m3_split_hi(vh);
-        lo[j] = part ? vl - hl : hl;
-        hi[j] = part ? vh - hh : hh;
-      }
-      f.x = pack_e4m3x4(lo[0], lo[1], lo[2], lo[3]);
-      f.y = pack_e4m3x4(hi[0], hi[1], hi[2], hi[3]);
-    }
-    frag[i] = f;
-  }
-  named_bar(kBarConsumers, kConsumers);
 }
 
-// One 16-row unit over n_groups block groups: acc[quad][r] with r = (row g,
-// split 0), (row g, split 1), (row g+8, split 0), (row g+8, split 1) of token
-// 4 * quad + c, in units of 2^(s_t - 9).  Four block tiles per group are
-// staged: loads, code masking, one m16n8k32 MMA per quad (accumulator started
-// at the block's correction), then the fp16 block scales.
-// Block groups [grp0, grp1) of a unit whose K spans n_groups groups; adds to acc.
-template <int NQ>
-__device__ __forceinline__ void unit_gemv(const uint8_t *st, int grp0, int grp1, int n_groups, const uint2 *frag,
-                                          const float *corr, int lane, float (&acc)[2][4]) {
+// Block groups [grp0, grp1) of one 16-row unit against the (at most 8) token
+// rows `rows` (row g of this lane's B column; tokens >= T read the zero row `zrow`); adds
+// to acc = (row g, token 2c), (row g, token 2c+1), (row g+8, token 2c),
+// (row g+8, token 2c+1).  Per block: the codes decode to bf16 128 + q /
+// 128 + 4q (decode_q2_biased), two m16n8k16 MMAs with the accumulator started
+// at the block's corr, then the fp16 block scales.
+__device__ __forceinline__ void unit_gemv(const uint8_t *st, int grp0, int grp1, const uint16_t *rows, int stride,
+                                          int T, const uint16_t *zrow, const float *corr, int lane, float (&acc)[4]) {
   const int g = lane >> 2, c = lane & 3;
-  const int nb = n_groups * 4;
+  const uint16_t *xrow = (g < T ? rows + g * stride : zrow) + 4 * c;
   for (int grp = grp0; grp < grp1; ++grp) {
     const uint8_t *gp = st + (size_t)grp * kGroupBytes;
     const uint4 cw = lds128(gp + lane * 16);
     const uint4 sw = lds128(gp + kGroupCodeBytes + g * 16);
     const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
     const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
-    uint2 bf[NQ][4];
-    float cn[NQ][4];
+    uint2 b0[4], b1[4];
+    float2 nc[4];
 #pragma unroll
     for (int blk = 0; blk < 4; ++blk) {
       const int b = grp * 4 + blk;
-#pragma unroll
-      for (int qd = 0; qd < NQ; ++qd) {
-        bf[qd][blk] = frag[(qd * nb + b) * 32 + lane];
-        cn[qd][blk] = corr[b * kMaxTok + 4 * qd + c];
-      }
+      b0[blk] = *reinterpret_cast<const uint2 *>(xrow + 32 * b);
+      b1[blk] = *reinterpret_cast<const uint2 *>(xrow + 32 * b + 16);
+      nc[blk] = *reinterpret_cast<const float2 *>(corr + b * kMaxTok + 2 * c);
     }
-    float d[NQ][4][4];
+    uint32_t p[4][8];
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) decode_q2_biased(cws[blk], p[blk]);
+    float d[4][4];
 #pragma unroll
     for (int blk = 0; blk < 4; ++blk) {
-      uint32_t am[4];
-      decode_q2_e4m3(cws[blk], am);
+      const uint32_t a0[4] = {p[blk][0], p[blk][1], p[blk][2], p[blk][3]};
+      const float cin[4] = {nc[blk].x, nc[blk].y, nc[blk].x, nc[blk].y};
+      mma_bf16_16816(d[blk], a0, b0[blk].x, b0[blk].y, cin);
+    }
 #pragma unroll
-      for (int qd = 0; qd < NQ; ++qd) {
-        const float cin[4] = {cn[qd][blk], 0.f, cn[qd][blk], 0.f};
-        mma_e4m3_16832(d[qd][blk], am, bf[qd][blk].x, bf[qd][blk].y, cin);
-      }
+    for (int blk = 0; blk < 4; ++blk) {
+      const uint32_t a1[4] = {p[blk][4], p[blk][5], p[blk][6], p[blk][7]};
+      mma_bf16_16816(d[blk], a1, b1[blk].x, b1[blk].y, d[blk]);
     }
 #pragma unroll
     for (int blk = 0; blk < 4; ++blk) {
       const float2 s2 = __half22float2(*reinterpret_cast<const __half2 *>(&sws[blk]));
-#pragma unroll
-      for (int qd = 0; qd < NQ; ++qd) {
-        fma2_bcast(acc[qd][0], acc[qd][1], s2.x, d[qd][blk][0], d[qd][blk][1]);
-        fma2_bcast(acc[qd][2], acc[qd][3], s2.y, d[qd][blk][2], d[qd][blk][3]);
-      }
+      fma2_bcast(acc[0], acc[1], s2.x, d[blk][0], d[blk][1]);
+      fma2_bcast(acc[2], acc[3], s2.y, d[blk][2], d[blk][3]);
     }
   }
 }
@@ -252,12 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const SmemLayout L = smem_layout(T, H, a.ns, a.stage_bytes);
   uint16_t *xs = reinterpret_cast<uint16_t *>(smem + L.xs);
   float *corr = reinterpret_cast<float *>(smem + L.corr);
-  uint2 *xb = reinterpret_cast<uint2 *>(smem + L.xb);
-  float *xsc = reinterpret_cast<float *>(smem + L.xsc);
-  uint2 *hb = reinterpret_cast<uint2 *>(smem + L.hb);
   float *hcorr = reinterpret_cast<float *>(smem + L.hcorr);
-  float *hsc = reinterpret_cast<float *>(smem + L.hsc);
-  const int nq = token_quads(T);
   float *rpart = reinterpret_cast<float *>(smem + L.rpart);
   float *red = reinterpret_cast<float *>(smem + L.red);
   int *sel_idx = reinterpret_cast<int *>(smem + L.sel_idx);
@@ -274,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const int xstride = H + 16;
+  const uint16_t *zrow = xs + T * xstride;  // zeros: the B column of tokens >= T
   const int n_rrows = E > (int)blockIdx.x ? (E - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   float *wr_s = reinterpret_cast<float *>(ring);  // router rows live in the ring until phase C
 
@@ -300,14 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       for (size_t o = 0; o < n; o += 32768) bulk_prefetch_l2(a.shared + off + o, (uint32_t)min((size_t)32768, n - o));
     }
   }
+  for (int i = tid; i < xstride / 8; i += kConsumers)
+    reinterpret_cast<uint4 *>(xs + T * xstride)[i] = make_uint4(0u, 0u, 0u, 0u);
   {
     if (blockIdx.x == 0)
       for (int i = tid; i < G.dn_units + kMaxEntries; i += kConsumers) a.tile_cnt[i] = 0u;
-    cp_async_wait_group<1>();  // this thread's token pieces have landed
-    named_bar(kBarConsumers, kConsumers);
-    // Tokens as e4m3 B fragments: per-token power-of-two scale, two split terms.
-    build_b_fragments(xs, xstride, H, T, nq, xb, corr, xsc, misc + 8, warp, lane, tid);
-    cp_async_wait_group<0>();  // router rows
+    cp_async_wait_group<0>();  // this thread's pieces of the tokens and router rows have landed
     named_bar(kBarConsumers, kConsumers);
     constexpr int kRowsPerPass = kConsumerWarps / kRouterParts;  // one warp per router row part
     for (int r0 = 0; r0 < n_rrows; r0 += kRowsPerPass) {
@@ -331,7 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       }
       named_bar(kBarConsumers, kConsumers);
     }
-    grid_barrier(a.gbar, kBarConsumers, kConsumers, tid == 0, a.status, &misc[2]);
+    // Arrive on the grid barrier, prepare the token rows as the B operand while the other CTAs finish
+    // their logits (the router is done with them), then wait.
+    const uint64_t bar_target = grid_arrive(a.gbar, kBarConsumers, kConsumers, tid == 0);
+    prep_rows(xs, xstride, H, T, corr, tid);
+    grid_wait(a.gbar, bar_target, kBarConsumers, kConsumers, tid == 0, a.status, &misc[2]);
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
     // All logits into shared memory first (one coalesced pass through L2), then one warp per token.
@@ -416,77 +357,75 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   // Stage s belongs to warp s % nw, which copies it (cp.async) into its own
   // ring slot, waits for its own copies, computes it and refills the slot with
   // its next stage s + nw.  No other warp touches the slot.
-  const int nw = a.nw, spw = 1;
+  const int nw = a.nw;
   auto expert_ptr = [&](int entry) -> const uint8_t * {
     const int e = ent[entry];
     return e == E ? a.shared : a.experts + (size_t)e * G.expert_bytes;
   };
-  auto stage_ptr = [&](int s) { return ring + (size_t)(warp * spw + (s / nw) % spw) * a.stage_bytes; };
-  // A stage is copied as 4 commit groups (its quarters, in order) so that the
-  // warp can start on the first quarter while the rest is still arriving:
-  // gate/up = one unit (quarter = 4 block groups), down = 2 units of 16 rows
-  // (quarter = half a unit).  Past the last stage the groups are empty.
-  auto issue_stage = [&](int s) {
-    for (int qt = 0; qt < 4; ++qt) {
-      if (s < n_st) {
-        uint8_t *dst = stage_ptr(s);
-        if (s < n_gu_st) {
-          const int id = g0 + s;
-          const size_t qb = G.gu_unit_bytes / 4;
-          warp_cp_async(dst + qt * qb,
-                        expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes + qt * qb,
-                        (uint32_t)qb, lane);
-        } else {
-          const int q = d0 + (s - n_gu_st) * pps + (qt >> 1);
-          const size_t hb2 = G.dn_unit_bytes / 2;
-          if (q < d1)
-            warp_cp_async(dst + (size_t)(qt >> 1) * G.dn_unit_bytes + (qt & 1) * hb2,
-                          expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes +
-                              (qt & 1) * hb2,
-                          (uint32_t)hb2, lane);
-        }
+  auto stage_ptr = [&](int) { return ring + (size_t)warp * a.stage_bytes; };
+  // A stage is copied as 4 commit groups (its quarters): gate/up = one unit
+  // (quarter = 4 block groups), down = 2 units of 16 rows (quarter = half a
+  // unit).  A warp walks the quarters of its stages in order and keeps the next
+  // two in flight: quarter i is computed after quarter i + 1 was issued, and
+  // quarter i + 2 goes into the slot region quarter i - 2 used.  Past the last
+  // stage the groups are empty.
+  auto issue_quarter = [&](int qi) {
+    const int s = warp + (qi >> 2) * nw, qt = qi & 3;
+    if (s < n_st) {
+      uint8_t *dst = stage_ptr(s);
+      if (s < n_gu_st) {
+        const int id = g0 + s;
+        const size_t qb = G.gu_unit_bytes / 4;
+        warp_cp_async(dst + qt * qb,
+                      expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes + qt * qb,
+                      (uint32_t)qb, lane);
+      } else {
+        const int q = d0 + (s - n_gu_st) * pps + (qt >> 1);
+        const size_t hb2 = G.dn_unit_bytes / 2;
+        if (q < d1)
+          warp_cp_async(dst + (size_t)(qt >> 1) * G.dn_unit_bytes + (qt & 1) * hb2,
+                        expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes +
+                            (qt & 1) * hb2,
+                        (uint32_t)hb2, lane);
       }
-      cp_async_commit();
     }
+    cp_async_commit();
   };
-  // quarter qt of the warp's current stage has landed (spw == 1: nothing newer is in flight)
-  auto wait_quarter = [&](int qt) {
-    if (qt == 0)
-      cp_async_wait_group<3>();
-    else if (qt == 1)
-      cp_async_wait_group<2>();
-    else if (qt == 2)
-      cp_async_wait_group<1>();
-    else
-      cp_async_wait_group<0>();
+  // Quarter qi has landed (only quarter qi + 1 may still be in flight), then queue quarter qi + 2.
+  int qi = 0;
+  auto next_quarter = [&]() {
+    cp_async_wait_group<1>();
     __syncwarp();
   };
-  if (warp < nw) issue_stage(warp);
+  auto done_quarter = [&]() {
+    __syncwarp();  // every lane has read the quarter before its region is refilled
+    issue_quarter(qi + 2);
+    ++qi;
+  };
+  if (warp < nw) {
+    issue_quarter(0);
+    issue_quarter(1);
+  }
 
   // ---------------- consumers, phase C: gate/up + SwiGLU ----------------
   for (int s_idx = warp; warp < nw && s_idx < n_gu_st; s_idx += nw) {
     const uint8_t *st = stage_ptr(s_idx);
-    float acc[2][4] = {};
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int gq = G.gu_groups / 4;  // block groups per quarter
     for (int qt = 0; qt < 4; ++qt) {
-      wait_quarter(qt);
-      if (nq == 1)
-        unit_gemv<1>(st, qt * gq, (qt + 1) * gq, G.gu_groups, xb, corr, lane, acc);
-      else
-        unit_gemv<2>(st, qt * gq, (qt + 1) * gq, G.gu_groups, xb, corr, lane, acc);
+      next_quarter();
+      unit_gemv(st, qt * gq, (qt + 1) * gq, xs, xstride, T, zrow, corr, lane, acc);
+      done_quarter();
     }
-    __syncwarp();
-    issue_stage(s_idx + spw * nw);
     const int id = g0 + s_idx;
     const int entry = id / G.gu_units, u = id % G.gu_units;
     const int i = 8 * u + g;  // tile rows g (gate) and g+8 (up) share intermediate row i
 #pragma unroll
-    for (int qd = 0; qd < 2; ++qd) {
-      const int n = 4 * qd + c;  // this lane's token
-      if (qd < nq && n < T) {
+    for (int hf = 0; hf < 2; ++hf) {
+      const int n = 2 * c + hf;  // this lane's tokens: 2c, 2c + 1
+      if (n < T) {
         const int j = tokj[entry * kMaxTok + n];
-        const float gate = (acc[qd][0] + acc[qd][1]) * xsc[n], up = (acc[qd][2] + acc[qd][3]) * xsc[n];
-        if (j >= 0) a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(gate) * up);
+        if (j >= 0) a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(acc[hf]) * acc[2 + hf]);
       }
     }
   }
@@ -527,43 +466,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     *reinterpret_cast<uint4 *>(hc + (he * T + t) * hstride + c8 * 8) = v;
   }
   named_bar(kBarConsumers, kConsumers);
-  for (int he = 0; he < n_hc; ++he)
-    build_b_fragments(hc + he * T * hstride, hstride, I, T, nq, hb + he * nq * (kMaxI / 32) * 32,
-                      hcorr + he * (kMaxI / 32) * kMaxTok, hsc + he * kMaxTok, misc + 8, warp, lane, tid);
+  for (int he = 0; he < n_hc; ++he) prep_rows(hc + he * T * hstride, hstride, I, T, hcorr + he * (kMaxI / 32) * kMaxTok, tid);
+  named_bar(kBarConsumers, kConsumers);
 
   for (int s_idx = n_gu_st + ((warp - n_gu_st % nw + nw) % nw); warp < nw && s_idx < n_st; s_idx += nw) {
     const int sd = s_idx - n_gu_st;
     const uint8_t *st = stage_ptr(s_idx);
     const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
-    for (int q = q0; q < q1; ++q) {
+    for (int q = q0; q < q0 + pps; ++q) {  // a stage always spans 4 quarters, the last one may hold one unit
+      const bool live = q < q1;
       const int entry = q / G.dn_units, tile = q % G.dn_units, he = entry - e_lo;
       const uint8_t *pp_st = st + (size_t)(q - q0) * G.dn_unit_bytes;
-      const uint2 *hbe = hb + he * nq * (kMaxI / 32) * 32;
+      const uint16_t *hrows = hc + he * T * hstride;
       const float *hce = hcorr + he * (kMaxI / 32) * kMaxTok;
-      float acc[2][4] = {};
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
       const int hg = G.dn_groups / 2;  // block groups per half unit
       for (int h2 = 0; h2 < 2; ++h2) {
-        wait_quarter(2 * (q - q0) + h2);
-        if (nq == 1)
-          unit_gemv<1>(pp_st, h2 * hg, (h2 + 1) * hg, G.dn_groups, hbe, hce, lane, acc);
-        else
-          unit_gemv<2>(pp_st, h2 * hg, (h2 + 1) * hg, G.dn_groups, hbe, hce, lane, acc);
+        next_quarter();
+        if (live) unit_gemv(pp_st, h2 * hg, (h2 + 1) * hg, hrows, hstride, T, zrow, hce, lane, acc);
+        done_quarter();
       }
-      // partial tile layout: lane (g, c) -> {row g tok c, row g+8 tok c, row g tok c+4, row g+8 tok c+4}
-      float o4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int qd = 0; qd < 2; ++qd) {
-        if (qd >= nq) break;
-        const int n = 4 * qd + c;
-        const float f = hsc[he * kMaxTok + n] * tokw[entry * kMaxTok + n];
-        o4[2 * qd] = (acc[qd][0] + acc[qd][1]) * f;
-        o4[2 * qd + 1] = (acc[qd][2] + acc[qd][3]) * f;
-      }
+      if (!live) continue;
+      // partial tile layout: lane (g, c) -> {row g tok 2c, row g tok 2c+1, row g+8 tok 2c, row g+8 tok 2c+1}
+      const float w0 = 2 * c < T ? tokw[entry * kMaxTok + 2 * c] : 0.f;
+      const float w1 = 2 * c + 1 < T ? tokw[entry * kMaxTok + 2 * c + 1] : 0.f;
+      const float o4[4] = {acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1};
       float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
       *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
     }
-    __syncwarp();
-    issue_stage(s_idx + spw * nw);
   }
   cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
 
@@ -607,11 +537,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     }
     const int r0 = 16 * tile + g;
 #pragma unroll
-    for (int qd = 0; qd < 2; ++qd) {
-      const int n = 4 * qd + c;
+    for (int hf = 0; hf < 2; ++hf) {
+      const int n = 2 * c + hf;
       if (n < T) {
-        a.out[(size_t)n * H + r0] = float_to_bf16_bits(o[2 * qd]);
-        a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 * qd + 1]);
+        a.out[(size_t)n * H + r0] = float_to_bf16_bits(o[hf]);
+        a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 + hf]);
       }
     }
   }

@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(128) router_logits_mma_kernel(const uint16_t *
 __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int T, int E, int k,
                                                    int32_t *__restrict__ idx, float *__restrict__ w,
                                                    uint32_t *bitmap, int words) {
-  __shared__ uint64_t scratch[8][64];
+  __shared__ __align__(16) uint64_t scratch[8][64];
   const int t = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;

@@ -162,51 +162,65 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Top-k by threshold, filter and rank (E <= 32 * NPL, one warp).  Each
-// (logit, index) becomes a 64-bit value key << 32 | ~index, so that "larger"
-// is the selection order (logit desc, index asc).  The k-th largest of the 32
-// lane maxima bounds the k-th largest overall from below; the values at or
-// above it (usually a few more than k) are compacted one per lane and ranked
-// by counting.  Falls back to warp_topk_regs when more than 32 values pass.
-// `scratch` is 64 uint64 of shared memory private to the warp.  Same
-// selection and softmax as warp_topk, hence the same result.
+// Top-k by threshold, filter and rank (E <= 32 * NPL, one warp).  Every
+// (logit, index) is ranked by the 64-bit key float_key(logit) << 32 | ~index,
+// so that "larger" is the selection order (logit desc, index asc).  The k-th
+// largest of the 32 lane maxima, L, bounds the k-th largest value from below;
+// the values at or above it (usually a few more than k) are compacted into
+// shared memory and ranked by counting.  Falls back to warp_topk_regs when
+// more than 32 values pass.  Few dependent steps: shared-memory broadcasts
+// instead of shuffle chains.  `scratch` is 64 uint64 of shared memory private
+// to the warp.  Same selection and softmax as warp_topk, hence the same result.
 template <int NPL, bool kSmem = false>
 __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, int lane, uint64_t *scratch,
                                                int &e_out, float &w_out) {
-  uint64_t v[NPL];
-  uint64_t m = 0;
+  uint32_t kv[NPL];
+  uint32_t mk = 0;
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
     const int e = lane + 32 * j;
-    v[j] = e < E ? ((uint64_t)float_key(load_logit<kSmem>(row, e)) << 32) | (uint32_t)~e : 0ull;
-    m = v[j] > m ? v[j] : m;
+    kv[j] = e < E ? float_key(load_logit<kSmem>(row, e)) : 0u;
+    mk = kv[j] > mk ? kv[j] : mk;
   }
-  int rank = 0;
-#pragma unroll 8
-  for (int o = 0; o < 32; ++o) rank += __shfl_sync(0xffffffffu, m, o) > m;
-  const uint32_t sel = __ballot_sync(0xffffffffu, rank == k - 1);
-  const uint64_t L = __shfl_sync(0xffffffffu, m, __ffs(sel) - 1);
+  uint32_t *lmax = reinterpret_cast<uint32_t *>(scratch + 32);  // 32 lane maxima
+  lmax[lane] = mk;
+  __syncwarp();
+  int ge = 0;  // lane maxima >= mine
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 q = reinterpret_cast<const uint4 *>(lmax)[i];
+    ge += (q.x >= mk) + (q.y >= mk) + (q.z >= mk) + (q.w >= mk);
+  }
+  // L = the k-th largest lane maximum: the largest mk that at least k lane maxima reach
+  const uint32_t L = __reduce_max_sync(0xffffffffu, ge >= k ? mk : 0u);
   int cnt = 0;
 #pragma unroll
-  for (int j = 0; j < NPL; ++j) cnt += v[j] >= L;
+  for (int j = 0; j < NPL; ++j) cnt += kv[j] >= L;
   const int total = __reduce_add_sync(0xffffffffu, cnt);
   if (total > 32) {
     __syncwarp();
     warp_topk_regs<NPL, kSmem>(row, E, k, lane, e_out, w_out);
     return;
   }
-  int base = 0;
+  int pos = cnt;  // exclusive prefix of the candidate counts
 #pragma unroll
-  for (int j = 0; j < NPL; ++j) {
-    const bool p = v[j] >= L;
-    const uint32_t bal = __ballot_sync(0xffffffffu, p);
-    if (p) scratch[base + __popc(bal & ((1u << lane) - 1u))] = v[j];
-    base += __popc(bal);
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, pos, off);
+    if (lane >= off) pos += v;
   }
+  pos -= cnt;
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < NPL; ++j)
+    if (kv[j] >= L) scratch[pos++] = ((uint64_t)kv[j] << 32) | (uint32_t)~(lane + 32 * j);
   __syncwarp();
   const uint64_t cand = lane < total ? scratch[lane] : 0ull;
   int r = 0;
-  for (int o = 0; o < total; ++o) r += scratch[o] > cand;
+#pragma unroll
+  for (int o = 0; o < 32; o += 2) {
+    const ulonglong2 q = reinterpret_cast<const ulonglong2 *>(scratch)[o >> 1];
+    r += (o < total && q.x > cand) + (o + 1 < total && q.y > cand);
+  }
   __syncwarp();
   if (lane < total && r < k) scratch[32 + r] = cand;
   __syncwarp();

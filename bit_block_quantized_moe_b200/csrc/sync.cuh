@@ -127,18 +127,28 @@ __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
 
 // Grid-wide barrier for a co-resident (cooperatively launched) grid, over one
 // monotonic 64-bit arrival counter (zeroed once with the workspace, never
-// reset).  The participating threads of each CTA meet at named barrier
-// `bar_id`; thread `leader` fences, adds 1 and waits until the counter reaches
-// the next multiple of gridDim.x: one atomic round trip per CTA.  Returns false
-// (and sets the status timeout bit) if the wait hit the limit.
-__device__ __forceinline__ bool grid_barrier(uint64_t *count, int bar_id, int nthreads, bool leader, uint32_t *status,
-                                             int *flag_smem) {
+// reset), split in two so that independent work can run between arriving and
+// waiting.  grid_arrive: the participating threads of each CTA meet at named
+// barrier `bar_id`; thread `leader` fences, adds 1 and returns the count the
+// wait must reach (the next multiple of gridDim.x).  grid_wait: the leader
+// polls until the counter reaches it, then the threads meet again.  One atomic
+// round trip per CTA.  grid_wait returns false (and sets the status timeout
+// bit) if the wait hit the limit.
+__device__ __forceinline__ uint64_t grid_arrive(uint64_t *count, int bar_id, int nthreads, bool leader) {
   named_bar(bar_id, nthreads);
+  uint64_t target = 0;
   if (leader) {
-    bool ok = true;
     __threadfence();
     const unsigned long long old = atomicAdd(reinterpret_cast<unsigned long long *>(count), 1ull);
-    const uint64_t target = (old / gridDim.x + 1) * gridDim.x;
+    target = (old / gridDim.x + 1) * gridDim.x;
+  }
+  return target;
+}
+
+__device__ __forceinline__ bool grid_wait(const uint64_t *count, uint64_t target, int bar_id, int nthreads,
+                                          bool leader, uint32_t *status, int *flag_smem) {
+  if (leader) {
+    bool ok = true;
     const uint64_t t0 = global_timer_ns();
     while (ld_acquire_gpu_u64(count) < target) {
       if (global_timer_ns() - t0 > kWaitLimitNs) {
