@@ -54,6 +54,41 @@ def parse():
     return ap.parse_args()
 
 
+# Sources the fused decode kernel is compiled from; an ncu summary under profiles/ records
+# their hash, and its DRAM traffic is reported only while the sources still match.
+DECODE_SOURCES = ["decode.cu", "common.cuh", "sync.cuh", "router.cuh", "kernels.cuh"]
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_fused_kernel_t3.md")
+
+
+def decode_source_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "bit_block_quantized_moe_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_decode_traffic():
+    """(bytes per launch, note) from the committed ncu summary if it was taken on these sources, else (None, why)."""
+    try:
+        text = open(DECODE_PROFILE).read()
+    except OSError:
+        return None, "no ncu summary"
+    src = traffic = None
+    for line in text.splitlines():
+        if line.startswith("sources sha256:"):
+            src = line.split(":", 1)[1].strip()
+        if line.startswith("dram bytes per launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    if src is None or traffic is None:
+        return None, "summary lacks hash or traffic"
+    if src != decode_source_hash():
+        return None, "kernel changed since the ncu capture"
+    return traffic, "ncu dram__bytes_read.sum + dram__bytes_write.sum, " + os.path.basename(DECODE_PROFILE)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -327,6 +362,7 @@ def run_ours(args, world, rank, local):
     kern_ms = traced_kernel_ms(step, n_trace, M.MOE_KERNEL["decode_fused"], stream)
     hbm_peak = float(peaks["hbm_gbs"])
     kern_gbs = layer_bytes / (kern_ms * 1e-3) / 1e9
+    traffic, traffic_note = profiled_decode_traffic()
     layer_gbs = layer_bytes / (ms_per_step * 1e-3) / 1e9
 
     # ---- end to end through the public API, host buffers --------------------------------
@@ -390,7 +426,8 @@ def run_ours(args, world, rank, local):
             "peak": hbm_peak,
             "unit": "GB/s",
             "frac": kern_gbs / hbm_peak,
-            "traffic": None,
+            "traffic": traffic,
+            "traffic_source": traffic_note,
             "peak_source": f"{peak_src} hbm_gbs",
             "kernel_ms": kern_ms,
             "algorithmic_bytes": layer_bytes,

@@ -38,7 +38,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   };
   const size_t o_hdr = take(256);                          // status, counters
   const size_t o_bitmap = take((size_t)E * words * 4);    // cleared each call, together with the counters below
-  const size_t o_zero_tail = take(256);                    // done counter lives here
+  const size_t o_zero_tail = take(256);                    // end of the range the router clears
   const size_t o_wprefix = take((size_t)E * words * 4);
   const size_t o_counts = take((size_t)E * 4);
   const size_t o_offsets = take((size_t)(E + 1) * 4);
@@ -64,7 +64,6 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->n_items = reinterpret_cast<uint32_t *>(b + o_hdr + 4);
     ws->bitmap = reinterpret_cast<uint32_t *>(b + o_bitmap);
     ws->zero_begin = ws->bitmap;
-    ws->done_counter = reinterpret_cast<uint32_t *>(b + o_zero_tail);
     ws->zero_words = (o_zero_tail + 4 - o_bitmap) / 4;
     ws->wprefix = reinterpret_cast<uint32_t *>(b + o_wprefix);
     ws->counts = reinterpret_cast<int32_t *>(b + o_counts);

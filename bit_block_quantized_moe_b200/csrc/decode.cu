@@ -1,30 +1,30 @@
 // Fused decode/verify-window layer (T <= 8 tokens) in one persistent,
-// cooperatively launched kernel (sm_100a).  One CTA per SM: 14 consumer
-// warps and 1 producer warp.
+// cooperatively launched kernel (sm_100a).  One CTA per SM, 14 warps, each of
+// which both streams and computes.
 //
-//  A  The producer warp copies (cp.async, 16 B per lane) the tokens and this
-//     CTA's router rows into shared memory and prefetches its slice of the
-//     shared expert into L2.  Consumers compute the router rows (2 warps per row, one
-//     half of K each) and the correction sums of the biased decode.
-//     -- grid barrier: all logits written (the token fragments are built
-//        between arriving and waiting) --
-//  B  Every CTA selects the top-k of every token (threshold + rank, one warp
-//     per token) and builds the same sorted list of touched experts plus the
-//     shared expert.
+//  A  Every thread copies (cp.async, 16 B) its pieces of the tokens and of this
+//     CTA's router rows into shared memory; one thread prefetches the CTA's
+//     slice of the shared expert into L2.  2 warps per router row (one half of
+//     K each) write the logits.
+//     -- grid barrier: all logits written.  Between arriving and waiting the
+//        CTA prepares its token rows as the MMA B operand (block correction
+//        sums, the (4c+2, 4c+3) pairs scaled by 1/4) --
+//  B  All logits into shared memory; one warp per token selects the top-k
+//     (threshold + rank) and the CTA builds the same sorted list of touched
+//     experts plus the shared expert as every other CTA.
 //  C  Work lists, expert-major, cut into equal contiguous ranges per CTA:
-//     gate/up units (expert, 8 intermediate rows) and down pairs (expert, 16
-//     output rows).  The producer streams the CTA's units into a ring of
-//     shared-memory stages as stages free up; stage s belongs to consumer
-//     warp s % min(14, stages), which computes the whole unit (full K) with no cross-warp
-//     reduction and writes h = silu(g) * u (bf16) straight from its
-//     accumulators.  At the end the CTA publishes, per expert, how many of
+//     gate/up units (expert, 8 intermediate rows) and down stages (expert, two
+//     16-row units).  Stage s belongs to warp s % 14, which copies it into its
+//     own shared-memory slot in four cp.async groups, keeps the next two
+//     quarters in flight while it computes, runs the whole unit (full K) with
+//     no cross-warp reduction and writes h = silu(g) * u (bf16) straight from
+//     its accumulators.  At the end the CTA publishes, per expert, how many of
 //     its units are done.
 //  D  Once the h of the (at most two) experts in the CTA's down range is
 //     complete (per-expert counter, bounded wait) it is copied into shared
-//     memory; each down stage (up to 4 pairs) again belongs to one warp:
-//     partial = w[t, e] * (Wd_e h_e) per (expert, tile).  The last CTA to
-//     contribute to a tile sums its partials in expert order and writes out
-//     (bf16).
+//     memory; each down stage (two 16-row units) again belongs to one warp:
+//     partial = w[t, e] * (Wd_e h_e) per (expert, tile).  The warp that writes
+//     a tile's last partial sums them in expert order and writes out (bf16).
 // Dequantisation happens in registers: the 2-bit codes of a row OR into the
 // mantissa of bf16 128.0 (128 + q, or 128 + 4q with the matching activation
 // pair pre-scaled by 1/4), one logic op per pair of weights, and feed
@@ -469,50 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   for (int he = 0; he < n_hc; ++he) prep_rows(hc + he * T * hstride, hstride, I, T, hcorr + he * (kMaxI / 32) * kMaxTok, tid);
   named_bar(kBarConsumers, kConsumers);
 
-  for (int s_idx = n_gu_st + ((warp - n_gu_st % nw + nw) % nw); warp < nw && s_idx < n_st; s_idx += nw) {
-    const int sd = s_idx - n_gu_st;
-    const uint8_t *st = stage_ptr(s_idx);
-    const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
-    for (int q = q0; q < q0 + pps; ++q) {  // a stage always spans 4 quarters, the last one may hold one unit
-      const bool live = q < q1;
-      const int entry = q / G.dn_units, tile = q % G.dn_units, he = entry - e_lo;
-      const uint8_t *pp_st = st + (size_t)(q - q0) * G.dn_unit_bytes;
-      const uint16_t *hrows = hc + he * T * hstride;
-      const float *hce = hcorr + he * (kMaxI / 32) * kMaxTok;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int hg = G.dn_groups / 2;  // block groups per half unit
-      for (int h2 = 0; h2 < 2; ++h2) {
-        next_quarter();
-        if (live) unit_gemv(pp_st, h2 * hg, (h2 + 1) * hg, hrows, hstride, T, zrow, hce, lane, acc);
-        done_quarter();
-      }
-      if (!live) continue;
-      // partial tile layout: lane (g, c) -> {row g tok 2c, row g tok 2c+1, row g+8 tok 2c, row g+8 tok 2c+1}
-      const float w0 = 2 * c < T ? tokw[entry * kMaxTok + 2 * c] : 0.f;
-      const float w1 = 2 * c + 1 < T ? tokw[entry * kMaxTok + 2 * c + 1] : 0.f;
-      const float o4[4] = {acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1};
-      float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
-      *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
-    }
-  }
-  cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
-
-  // Count this CTA's contributions per output tile (one fence per writer
-  // warp); the last contributor of a tile sums its partials in expert order.
-  int *done_tiles = sel_idx;  // phase-B scratch, free now
-  __threadfence();
-  named_bar(kBarConsumers, kConsumers);
-  for (int i = tid; i < d1 - d0; i += kConsumers) {
-    const int tile = (d0 + i) % G.dn_units;
-    if (atomicAdd(&a.tile_cnt[tile], 1u) == (uint32_t)(nent - 1)) {
-      __threadfence();
-      done_tiles[atomicAdd(&misc[3], 1)] = tile;
-    }
-  }
-  named_bar(kBarConsumers, kConsumers);
-  const int n_done = misc[3];
-  for (int i = warp; i < n_done; i += kConsumerWarps) {
-    const int tile = done_tiles[i];
+  // Sums a finished output tile's partials in expert order (deterministic) and writes its rows.
+  auto reduce_tile = [&](int tile) {
     float o[4] = {0.f, 0.f, 0.f, 0.f};
     const float *pp = a.partial + (size_t)tile * 128 + lane * 4;
     int e2 = 0;
@@ -544,7 +502,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 + hf]);
       }
     }
+  };
+
+  for (int s_idx = n_gu_st + ((warp - n_gu_st % nw + nw) % nw); warp < nw && s_idx < n_st; s_idx += nw) {
+    const int sd = s_idx - n_gu_st;
+    const uint8_t *st = stage_ptr(s_idx);
+    const int q0 = d0 + sd * pps, q1 = min(d1, q0 + pps);
+    for (int q = q0; q < q0 + pps; ++q) {  // a stage always spans 4 quarters, the last one may hold one unit
+      const bool live = q < q1;
+      const int entry = q / G.dn_units, tile = q % G.dn_units, he = entry - e_lo;
+      const uint8_t *pp_st = st + (size_t)(q - q0) * G.dn_unit_bytes;
+      const uint16_t *hrows = hc + he * T * hstride;
+      const float *hce = hcorr + he * (kMaxI / 32) * kMaxTok;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int hg = G.dn_groups / 2;  // block groups per half unit
+      for (int h2 = 0; h2 < 2; ++h2) {
+        next_quarter();
+        if (live) unit_gemv(pp_st, h2 * hg, (h2 + 1) * hg, hrows, hstride, T, zrow, hce, lane, acc);
+        done_quarter();
+      }
+      if (!live) continue;
+      // partial tile layout: lane (g, c) -> {row g tok 2c, row g tok 2c+1, row g+8 tok 2c, row g+8 tok 2c+1}
+      const float w0 = 2 * c < T ? tokw[entry * kMaxTok + 2 * c] : 0.f;
+      const float w1 = 2 * c + 1 < T ? tokw[entry * kMaxTok + 2 * c + 1] : 0.f;
+      const float o4[4] = {acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1};
+      float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
+      *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+      // Count the contribution; the warp that brings the tile's last one sums all its
+      // partials in expert order right away and writes the output rows.
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(&a.tile_cnt[tile], 1u) == (uint32_t)(nent - 1);
+      }
+      if (__shfl_sync(0xffffffffu, last, 0)) {
+        __threadfence();
+        reduce_tile(tile);
+      }
+    }
   }
+
+  cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
 }
 
 }  // namespace

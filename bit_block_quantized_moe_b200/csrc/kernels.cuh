@@ -10,7 +10,6 @@ struct Workspace {
   uint32_t *status;        // sticky status word
   uint32_t *zero_begin;    // [zero_begin, zero_begin + zero_words) is cleared by the router kernel
   size_t zero_words;
-  uint32_t *done_counter;  // last-block counter of the dispatch scan (inside the zeroed range)
   uint32_t *n_items;
   uint32_t *bitmap;        // [E][words] token-membership bits per expert (inside the zeroed range)
   uint32_t *wprefix;       // [E][words] exclusive popcount prefix per word

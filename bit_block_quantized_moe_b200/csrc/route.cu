@@ -317,14 +317,49 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, 
 // independent of thread timing.  The shared expert's slots follow the routed
 // ones: position T*k + t.
 
-__global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__restrict__ bitmap, int words, int E,
-                                                            int T, int k, uint32_t *__restrict__ wprefix,
-                                                            int32_t *counts, int32_t *offsets, int4 *items,
-                                                            uint32_t *n_items, int4 *tc_items, uint32_t *n_tc_items,
-                                                            uint32_t *done_counter) {
+// One CTA of 1024 threads: per expert (one warp each, in turn) the popcount
+// prefix of its membership words and its count; then a block-wide exclusive
+// scan gives the offsets and the starts of each expert's work items (tiles of
+// 8 tokens for the register-dequant path, 64 for the tcgen05 path); the shared
+// expert's items follow the routed ones.
+constexpr int kScanThreads = 1024;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sums[lane];
+    int wi = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += t;
+    }
+    warp_sums[lane] = wi - ws;  // exclusive over warps
+    if (lane == 31) warp_sums[32] = wi;
+  }
+  __syncthreads();
+  const int r = warp_sums[warp] + incl - v;
+  total = warp_sums[32];
+  __syncthreads();  // warp_sums is reused by the next scan
+  return r;
+}
+
+__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(const uint32_t *__restrict__ bitmap, int words,
+                                                                     int E, int T, int k,
+                                                                     uint32_t *__restrict__ wprefix, int32_t *counts,
+                                                                     int32_t *offsets, int4 *items, uint32_t *n_items,
+                                                                     int4 *tc_items, uint32_t *n_tc_items) {
+  __shared__ int warp_sums[33];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (e < E) {
+  for (int e = warp; e < E; e += kScanThreads / 32) {
     uint32_t run = 0;
     for (int w0 = 0; w0 < words; w0 += 32) {
       const int wi = w0 + lane;
@@ -341,57 +376,37 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const uint32_t *__re
     }
     if (lane == 0) counts[e] = (int32_t)run;
   }
-  // The last block to finish turns counts into offsets and work items.
-  __shared__ bool is_last;
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(done_counter, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  // Work items: (expert, first sorted position, tokens) in tiles of 8 tokens
-  // (register-dequant path) and of 64 tokens (tcgen05 path).
-  __shared__ int s_cnt[256], s_items[256], s_tc[256];
-  const int per = (E + blockDim.x - 1) / blockDim.x;
+  // thread i owns experts [i * per, (i + 1) * per)
+  const int per = (E + kScanThreads - 1) / kScanThreads;
   const int eb = threadIdx.x * per, ee = min(E, eb + per);
   int my_cnt = 0, my_items = 0, my_tc = 0;
   for (int i = eb; i < ee; ++i) {
-    const int c = ((volatile int32_t *)counts)[i];
+    const int c = counts[i];
     my_cnt += c;
     my_items += (c + 7) >> 3;
     my_tc += (c + 63) >> 6;
   }
-  s_cnt[threadIdx.x] = my_cnt;
-  s_items[threadIdx.x] = my_items;
-  s_tc[threadIdx.x] = my_tc;
-  __syncthreads();
-  if (threadIdx.x == 0) {  // tiny serial scan over 256 partial sums
-    int a = 0, b = 0, tc = 0;
-    for (int i = 0; i < (int)blockDim.x; ++i) {
-      const int ca = s_cnt[i], cb = s_items[i], cc = s_tc[i];
-      s_cnt[i] = a;
-      s_items[i] = b;
-      s_tc[i] = tc;
-      a += ca;
-      b += cb;
-      tc += cc;
-    }
-    offsets[E] = a;  // == T * k
-    const int shared_items = (T + 7) >> 3;
-    for (int i = 0; i < shared_items; ++i) items[b + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
-    *n_items = (uint32_t)(b + shared_items);
-    const int shared_tc = (T + 63) >> 6;
-    for (int i = 0; i < shared_tc; ++i) tc_items[tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
-    *n_tc_items = (uint32_t)(tc + shared_tc);
-  }
-  __syncthreads();
-  int pos = s_cnt[threadIdx.x], it = s_items[threadIdx.x], itc = s_tc[threadIdx.x];
+  int tot_cnt, tot_items, tot_tc;
+  int pos = block_exclusive_scan(my_cnt, warp_sums, tot_cnt);
+  int it = block_exclusive_scan(my_items, warp_sums, tot_items);
+  int itc = block_exclusive_scan(my_tc, warp_sums, tot_tc);
   for (int i = eb; i < ee; ++i) {
-    const int c = ((volatile int32_t *)counts)[i];
+    const int c = counts[i];
     offsets[i] = pos;
     for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
     for (int j = 0; j < c; j += 64) tc_items[itc++] = make_int4(i, pos + j, min(64, c - j), 0);
     pos += c;
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = tot_cnt;  // == T * k when every index was valid
+    const int shared_items = (T + 7) >> 3;
+    for (int i = 0; i < shared_items; ++i) items[tot_items + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
+    *n_items = (uint32_t)(tot_items + shared_items);
+    const int shared_tc = (T + 63) >> 6;
+    for (int i = 0; i < shared_tc; ++i)
+      tc_items[tot_tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
+    *n_tc_items = (uint32_t)(tot_tc + shared_tc);
   }
 }
 
@@ -450,9 +465,8 @@ cudaError_t launch_dispatch_bits(const moe_dims &d, int T, const Workspace &ws, 
 cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s) {
   const int E = d.n_experts, k = d.top_k;
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, false, s);
-  dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, s>>>(ws.bitmap, ws.words, E, T, k, ws.wprefix, ws.counts, ws.offsets,
-                                                   ws.items, ws.n_items, ws.tc_items, ws.n_tc_items,
-                                                   ws.done_counter);
+  dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(ws.bitmap, ws.words, E, T, k, ws.wprefix, ws.counts, ws.offsets,
+                                                  ws.items, ws.n_items, ws.tc_items, ws.n_tc_items);
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, true, s);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
