@@ -1,17 +1,19 @@
 // Grouped expert GEMMs for prefill chunks on the 5th-generation tensor cores
 // (tcgen05, sm_100a).
 //
-// One persistent CTA per SM walks a list of work items (expert, 128-row M
-// tile, up to 64 tokens).  For each 128-wide K chunk:
-//   producer warp    : one TMA load of the tile's packed Q2 codes + scales (8
-//                      units x 640 B, a 4-D tensor map over the experts) and
+// One persistent CTA per SM walks a list of work items (expert, two 128-row
+// M tiles, up to 64 tokens): the two tiles share every load of the expert's
+// token rows.  For each 128-wide K chunk:
+//   producer warp    : one TMA load of both tiles' packed Q2 codes + scales
+//                      (16 units x 640 B, a 4-D tensor map over the experts;
+//                      units past the expert's last tile read as zeros) and
 //                      two of the expert's token rows (slot-sorted
 //                      activations, 128-byte swizzle, 16/32/64-row boxes)
-//                      into a shared-memory stage;
+//                      into one of 8 shared-memory stages;
 //   16 dequant warps : decode the codes in registers to bf16 d * (q - 1) and
 //                      store them into a tensor-memory A stage (tcgen05.st),
-//                      two blocks of one 16-row unit per warp;
-//   MMA warp        : 8 x tcgen05.mma (A from tensor memory, B from shared
+//                      one 16-row unit (4 blocks) per warp;
+//   MMA warp        : 2 x 8 tcgen05.mma (A from tensor memory, B from shared
 //                     memory), fp32 accumulators in tensor memory, commits
 //                     release the stages;
 //   4 epilogue warps: tcgen05.ld the accumulators; gate/up writes
@@ -28,17 +30,20 @@ namespace moe {
 
 namespace {
 
+constexpr int kMT = 2;             // 128-row M tiles per work item: they share every token-row load
 constexpr int kStages = 8;         // shared-memory stages (A codes + B rows)
-constexpr int kAStages = 6;        // tensor-memory A stages
+constexpr int kAStages = 2;        // tensor-memory A stages (kMT x 64 columns each)
 constexpr int kTileUnits = 8;      // 16-row units per 128-row M tile
 constexpr int kMaxN = 64;          // tokens per work item
-constexpr int kABytes = kTileUnits * kGroupBytes;  // 5120
-constexpr int kBSub = kMaxN * 128;                 // one 64-wide K half of the chunk: 8 KB
-constexpr int kStageBytes = kABytes + 2 * kBSub;   // 21504 (a multiple of 1024)
+constexpr int kABytes = kMT * kTileUnits * kGroupBytes;  // 10240
+constexpr int kBSub = kMaxN * 128;                       // one 64-wide K half of the chunk: 8 KB
+constexpr int kStageBytes = kABytes + 2 * kBSub;         // 26624 (a multiple of 1024)
 constexpr int kWarpProducer = 0, kWarpMMA = 1, kWarpDequant0 = 2, kNumDequant = 16, kWarpEpi0 = 18, kNumEpi = 4;
 constexpr int kThreadsTC = (kWarpEpi0 + kNumEpi) * 32;  // 704
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemA0 = 128;  // D buffers at columns 0 and 64; A stages at 128 + 64 * sa
+constexpr uint32_t kDCols = kMT * kMaxN;      // one accumulator buffer: kMT M tiles x 64 token columns
+constexpr uint32_t kTmemA0 = 2 * kDCols;      // D buffers at columns 0 and kDCols; A stages from 256
+static_assert(kTmemA0 + kAStages * kMT * 64 <= kTmemCols, "tensor memory columns");
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment for the 128-byte swizzle");
 
 struct TcArgs {
@@ -49,6 +54,7 @@ struct TcArgs {
   const int4 *items;          // (expert or E for shared, first sorted position, tokens <= 64, 0)
   const uint32_t *n_items;
   int mtiles;                 // 128-row tiles per expert for this projection
+  int mgroups;                // ceil(mtiles / kMT): work items per token item
   int kchunks;                // 128-wide K chunks (block groups)
   size_t unit_bytes;
   size_t sec_off;             // section offset inside a packed expert
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
   Bars &B = *reinterpret_cast<Bars *>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = (int)*a.n_items;
-  const int n_work = n_items * a.mtiles;
+  const int n_work = n_items * a.mgroups;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -129,8 +135,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
     if (lane == 0) {
       int cnt = 0;
       for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
-        const int4 it = a.items[w / a.mtiles];
-        const int mt = w % a.mtiles;
+        const int4 it = a.items[w / a.mgroups];
+        const int mt0 = (w % a.mgroups) * kMT;
         const int bsel = it.z <= 16 ? 0 : (it.z <= 32 ? 1 : 2);
         const int nrows = 16 << bsel;
         const CUtensorMap *amap = it.x == a.E ? &maps.a_shared : &maps.a_routed;
@@ -140,7 +146,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
           if (!waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) continue;
           uint8_t *st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&B.full[s], (uint32_t)(kABytes + 2 * nrows * 128));
-          tma_load_4d(st, amap, 0, kc, mt * kTileUnits, ae, &B.full[s]);
+          // kMT x 8 units; units past the expert's last tile read as zeros (tensor-map bounds)
+          tma_load_4d(st, amap, 0, kc, mt0 * kTileUnits, ae, &B.full[s]);
           for (int sub = 0; sub < 2; ++sub)
             tma_load_2d(st + kABytes + sub * kBSub, &maps.b[bsel], kc * 128 + sub * 64, it.y, &B.full[s]);
         }
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
     if (lane == 0) {
       int cnt = 0, acnt = 0, dcnt = 0;
       for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
-        const int4 it = a.items[w / a.mtiles];
+        const int4 it = a.items[w / a.mgroups];
         const int N = max(16, (it.z + 15) & ~15);
         const uint32_t idesc = umma_idesc_bf16(128, N);
         const int db = dcnt & 1;
@@ -165,10 +172,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
           tc_fence_after();
           const uint32_t bst = smem_u32(smem + s * kStageBytes + kABytes);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint64_t bdesc = umma_sdesc_sw128(bst + (j >> 2) * kBSub + (j & 3) * 32);
-            umma_ts(tbase + db * kMaxN, tbase + kTmemA0 + sa * 64 + 8 * j, bdesc, idesc, (kc | j) != 0);
-          }
+          for (int m = 0; m < kMT; ++m)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint64_t bdesc = umma_sdesc_sw128(bst + (j >> 2) * kBSub + (j & 3) * 32);
+              umma_ts(tbase + db * kDCols + m * kMaxN, tbase + kTmemA0 + (sa * kMT + m) * 64 + 8 * j, bdesc, idesc,
+                      (kc | j) != 0);
+            }
           umma_commit(&B.aempty[sa]);
           umma_commit(&B.empty[s]);
         }
@@ -180,9 +190,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       if (!mbar_wait(&B.done, 0)) set_status(a.status, kStatusTimeout);
     }
   } else if (warp < kWarpEpi0) {
-    // ---- dequant warps: 4 per TMEM lane quadrant = 2 units x 2 block pairs ----
+    // ---- dequant warps: 4 per TMEM lane quadrant = kMT (2) M tiles x 2 units, one whole unit each ----
     const int dw = warp - kWarpDequant0;
-    const int q = warp & 3, uq = (dw >> 2) & 1, bh = dw >> 3;
+    const int q = warp & 3, uq = (dw >> 2) & 1, m = dw >> 3;
     const int unit = 2 * q + uq;
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * uq) << 16;
     const int g = lane >> 2;
@@ -193,16 +203,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
         waitb(&B.aempty[sa], ((acnt / kAStages) & 1) ^ 1, B, a.status);
         tc_fence_after();
-        const uint8_t *gp = smem + s * kStageBytes + unit * kGroupBytes;
-        const uint2 cw = *reinterpret_cast<const uint2 *>(gp + lane * 16 + 8 * bh);
-        const uint2 sw = *reinterpret_cast<const uint2 *>(gp + kGroupCodeBytes + g * 16 + 8 * bh);
+        const uint8_t *gp = smem + s * kStageBytes + (m * kTileUnits + unit) * kGroupBytes;
+        const uint4 cw = *reinterpret_cast<const uint4 *>(gp + lane * 16);
+        const uint4 sw = *reinterpret_cast<const uint4 *>(gp + kGroupCodeBytes + g * 16);
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.empty[s]);  // this warp's share of the A codes is in registers
-        const uint32_t cws[2] = {cw.x, cw.y};
-        const uint32_t sws[2] = {sw.x, sw.y};
-        const uint32_t acol = tbase + lane_base + kTmemA0 + sa * 64 + 32 * bh;
+        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+        const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+        const uint32_t acol = tbase + lane_base + kTmemA0 + (sa * kMT + m) * 64;
 #pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
+        for (int bb = 0; bb < 4; ++bb) {
           uint32_t p[8];
           decode_q2_exact(cws[bb], p);
           uint32_t sg, sg8;
@@ -224,15 +234,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
     const int q = warp & 3;
     int dcnt = 0;
     for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
-      const int4 it = a.items[w / a.mtiles];
-      const int mt = w % a.mtiles;
+      const int4 it = a.items[w / a.mgroups];
+      const int mt0 = (w % a.mgroups) * kMT;
       const int db = dcnt & 1;
       waitb(&B.dfull[db], (dcnt >> 1) & 1, B, a.status);
       tc_fence_after();
       const int ntok = it.z;
+      for (int m = 0; m < kMT; ++m) {
+      const int mt = mt0 + m;
+      if (mt >= a.mtiles) break;  // the zero-filled tile past the expert's last one
       for (int col0 = 0; col0 < ntok; col0 += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + ((uint32_t)(32 * q) << 16) + db * kMaxN + col0, v);
+        tmem_ld_32x32b_x32(tbase + ((uint32_t)(32 * q) << 16) + db * kDCols + m * kMaxN + col0, v);
         tmem_wait_ld();
         const int nmax = min(32, ntok - col0);
         if (MODE == 0) {
@@ -252,6 +265,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
           for (int n = 0; n < 32; ++n)
             if (n < nmax) a.y_out[(size_t)(it.y + col0 + n) * H + row] = __uint_as_float(v[n]);
         }
+      }
       }
       tc_fence_before();
       __syncwarp();
@@ -304,14 +318,14 @@ bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols, int b
 }
 
 // 4-D map over packed units: (32-bit word within a 640-byte block group, group, unit, expert);
-// one box is one group of 8 consecutive units (5120 bytes, no swizzle).
+// one box is one group of 16 consecutive units (10240 bytes, no swizzle).
 bool make_units_map(CUtensorMap *map, const void *base, int groups, int units, int experts, size_t unit_bytes,
                     size_t expert_bytes) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {kGroupBytes / 4, (cuuint64_t)groups, (cuuint64_t)units, (cuuint64_t)experts};
   const cuuint64_t strides[3] = {kGroupBytes, unit_bytes, expert_bytes};
-  const cuuint32_t box[4] = {kGroupBytes / 4, 1, kTileUnits, 1};
+  const cuuint32_t box[4] = {kGroupBytes / 4, 1, kTileUnits * kMT, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -366,6 +380,7 @@ cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint
 
   // gate/up + SwiGLU: M = 2I interleaved rows (8 gate + 8 up per unit), K = H
   a.mtiles = G.gu_units / kTileUnits;
+  a.mgroups = (a.mtiles + kMT - 1) / kMT;
   a.kchunks = G.gu_groups;
   a.unit_bytes = G.gu_unit_bytes;
   a.sec_off = 0;
@@ -379,6 +394,7 @@ cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint
 
   // down: M = H rows, K = I
   a.mtiles = G.dn_units / kTileUnits;
+  a.mgroups = (a.mtiles + kMT - 1) / kMT;
   a.kchunks = G.dn_groups;
   a.unit_bytes = G.dn_unit_bytes;
   a.sec_off = G.gu_bytes;
