@@ -359,7 +359,34 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(const uint3
                                                                      int4 *tc_items, uint32_t *n_tc_items) {
   __shared__ int warp_sums[33];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = warp; e < E; e += kScanThreads / 32) {
+  constexpr int kNW = kScanThreads / 32;
+  if (words <= 32) {
+    // one word per lane: load 8 experts' words at once so their L2 round trips overlap
+    for (int e0 = warp; e0 < E; e0 += 8 * kNW) {
+      uint32_t bits[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = e0 + j * kNW;
+        bits[j] = (e < E && lane < words) ? bitmap[(size_t)e * words + lane] : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = e0 + j * kNW;
+        const uint32_t cnt = __popc(bits[j]);
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        if (e < E) {
+          if (lane < words) wprefix[(size_t)e * words + lane] = incl - cnt;
+          if (lane == 31) counts[e] = (int32_t)incl;
+        }
+      }
+    }
+  } else
+  for (int e = warp; e < E; e += kNW) {
     uint32_t run = 0;
     for (int w0 = 0; w0 < words; w0 += 32) {
       const int wi = w0 + lane;
@@ -489,7 +516,29 @@ __global__ void combine_kernel(const float *__restrict__ Y, const int32_t *__res
   if (i >= (long long)T * per_row) return;
   const int t = (int)(i / per_row), c4 = (int)(i % per_row);
   float4 acc = reinterpret_cast<const float4 *>(Y + ((size_t)T * k + t) * H)[c4];
-  for (int j = 0; j < k; ++j) {
+  // four slots' rows in flight at a time, accumulated in slot order
+  int j = 0;
+  for (; j + 4 <= k; j += 4) {
+    float4 v[4];
+    float wj[4];
+    bool ok[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int pos = slot_pos[(size_t)t * k + j + u];
+      ok[u] = pos >= 0;  // an invalid slot adds nothing
+      wj[u] = topk_w[(size_t)t * k + j + u];
+      v[u] = reinterpret_cast<const float4 *>(Y + (size_t)(ok[u] ? pos : 0) * H)[c4];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!ok[u]) continue;
+      acc.x = fmaf(wj[u], v[u].x, acc.x);
+      acc.y = fmaf(wj[u], v[u].y, acc.y);
+      acc.z = fmaf(wj[u], v[u].z, acc.z);
+      acc.w = fmaf(wj[u], v[u].w, acc.w);
+    }
+  }
+  for (; j < k; ++j) {
     const int pos = slot_pos[(size_t)t * k + j];
     if (pos < 0) continue;
     const float wj = topk_w[(size_t)t * k + j];
