@@ -10,17 +10,24 @@
 //                      two of the expert's token rows (slot-sorted
 //                      activations, 128-byte swizzle, 16/32/64-row boxes)
 //                      into one of 8 shared-memory stages;
-//   16 dequant warps : decode the codes in registers to bf16 d * (q - 1) and
-//                      store them into a tensor-memory A stage (tcgen05.st),
-//                      one 16-row unit (4 blocks) per warp;
-//   MMA warp        : 2 x 8 tcgen05.mma (A from tensor memory, B from shared
-//                     memory), fp32 accumulators in tensor memory, commits
-//                     release the stages;
+//   16 dequant warps : decode the codes in registers to bf16 d * (q - 1)
+//                      while the tensor core still reads the A stage they
+//                      will fill, then store them (tcgen05.st), one 16-row
+//                      unit (4 blocks) per warp; once the MMAs of a chunk
+//                      have completed they also release its shared-memory
+//                      stage to the producer;
+//   MMA warp        : 2 x 8 tcgen05.mma per chunk (A from tensor memory, B
+//                     from shared memory), fp32 accumulators in tensor
+//                     memory, one commit per chunk.  It waits only on the A
+//                     stage: the dequant warps passed the chunk's TMA barrier
+//                     before filling it, which orders the B rows too;
 //   4 epilogue warps: tcgen05.ld the accumulators; gate/up writes
-//                     h = silu(g) * u (bf16), down writes the fp32 expert
-//                     output rows for the combine.
-// Accumulators are double-buffered so the epilogue of one item overlaps the
-// MMAs of the next.  Every wait is bounded (sync.cuh).
+//                     h = silu(g) * u (bf16, each lane one SiLU per pair of
+//                     token columns), down writes the fp32 expert output rows
+//                     for the combine.
+// The issuing thread of the MMAs is the pipeline's pace: everything it waits
+// on is taken off its path.  Accumulators are double-buffered so the epilogue
+// of one item overlaps the MMAs of the next.  Every wait is bounded (sync.cuh).
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -70,6 +77,7 @@ struct Bars {
 };
 
 __device__ __forceinline__ bool waitb(uint64_t *bar, uint32_t parity, Bars &B, uint32_t *status) {
+  if (mbar_try_wait(bar, parity)) return true;
   if (*reinterpret_cast<volatile int *>(&B.abort)) return false;
   if (!mbar_wait(bar, parity)) {
     set_status(status, kStatusTimeout);
@@ -85,6 +93,9 @@ __device__ __forceinline__ void scale_pairs(uint32_t sh2, uint32_t &sg, uint32_t
   sg = pack_bf16x2(f.x, f.x);
   sg8 = pack_bf16x2(f.y, f.y);
 }
+
+// silu(z) = z / (1 + e^-z) with the fast division (h is rounded to bf16 right after).
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -111,7 +122,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&B.full[i], 1);
-      mbar_init(&B.empty[i], kNumDequant + 1);  // dequant warps read A, the MMA commit releases B
+      mbar_init(&B.empty[i], kNumDequant);  // each dequant warp, once the stage's MMAs have completed
     }
     for (int i = 0; i < kAStages; ++i) {
       mbar_init(&B.afull[i], kNumDequant);
@@ -157,7 +168,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
     }
   } else if (warp == kWarpMMA) {
     if (lane == 0) {
-      int cnt = 0, acnt = 0, dcnt = 0;
+      int cnt = 0, dcnt = 0;
       for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
         const int4 it = a.items[w / a.mgroups];
         const int N = max(16, (it.z + 15) & ~15);
@@ -165,22 +176,23 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         const int db = dcnt & 1;
         waitb(&B.dempty[db], ((dcnt >> 1) & 1) ^ 1, B, a.status);
         tc_fence_after();
-        for (int kc = 0; kc < a.kchunks; ++kc, ++cnt, ++acnt) {
-          const int s = cnt % kStages, sa = acnt % kAStages;
-          waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
-          waitb(&B.afull[sa], (acnt / kAStages) & 1, B, a.status);
+        const uint32_t dcol = tbase + db * kDCols;
+        for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
+          const int s = cnt % kStages, sa = cnt % kAStages;
+          // Every dequant warp waited on this chunk's TMA barrier before its arrival here, so the
+          // B rows of stage s are in shared memory as well.
+          waitb(&B.afull[sa], (cnt / kAStages) & 1, B, a.status);
           tc_fence_after();
-          const uint32_t bst = smem_u32(smem + s * kStageBytes + kABytes);
+          // K step j: 64-column half j / 4 of the stage's B rows, 32 bytes per step inside the half
+          const uint64_t bdesc0 = umma_sdesc_sw128(smem_u32(smem + s * kStageBytes + kABytes));
+          const uint32_t acol = tbase + kTmemA0 + sa * kMT * 64;
 #pragma unroll
           for (int m = 0; m < kMT; ++m)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint64_t bdesc = umma_sdesc_sw128(bst + (j >> 2) * kBSub + (j & 3) * 32);
-              umma_ts(tbase + db * kDCols + m * kMaxN, tbase + kTmemA0 + (sa * kMT + m) * 64 + 8 * j, bdesc, idesc,
-                      (kc | j) != 0);
-            }
+            for (int j = 0; j < 8; ++j)
+              umma_ts(dcol + m * kMaxN, acol + m * 64 + 8 * j,
+                      bdesc0 + (uint64_t)((j >> 2) * (kBSub >> 4) + (j & 3) * 2), idesc, (kc | j) != 0);
           umma_commit(&B.aempty[sa]);
-          umma_commit(&B.empty[s]);
         }
         umma_commit(&B.dfull[db]);
         ++dcnt;
@@ -196,32 +208,47 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
     const int unit = 2 * q + uq;
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * uq) << 16;
     const int g = lane >> 2;
-    int cnt = 0, acnt = 0;
+    int cnt = 0;
     for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
-      for (int kc = 0; kc < a.kchunks; ++kc, ++cnt, ++acnt) {
-        const int s = cnt % kStages, sa = acnt % kAStages;
+      for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
+        const int s = cnt % kStages, sa = cnt % kAStages;
         waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
-        waitb(&B.aempty[sa], ((acnt / kAStages) & 1) ^ 1, B, a.status);
-        tc_fence_after();
         const uint8_t *gp = smem + s * kStageBytes + (m * kTileUnits + unit) * kGroupBytes;
         const uint4 cw = *reinterpret_cast<const uint4 *>(gp + lane * 16);
         const uint4 sw = *reinterpret_cast<const uint4 *>(gp + kGroupCodeBytes + g * 16);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.empty[s]);  // this warp's share of the A codes is in registers
         const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
         const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
-        const uint32_t acol = tbase + lane_base + kTmemA0 + (sa * kMT + m) * 64;
+        // the whole unit in registers before the A stage is free: registers P0, P2 belong to row g,
+        // P1, P3 to row g+8
+        uint32_t av[4][8];
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
           uint32_t p[8];
           decode_q2_exact(cws[bb], p);
           uint32_t sg, sg8;
           scale_pairs(sws[bb], sg, sg8);
-          // registers P0, P2 belong to row g, P1, P3 to row g+8
-          tmem_st_16x256b(acol + 16 * bb, bf16x2_mul(p[0], sg), bf16x2_mul(p[2], sg), bf16x2_mul(p[1], sg8),
-                          bf16x2_mul(p[3], sg8));
-          tmem_st_16x256b(acol + 16 * bb + 8, bf16x2_mul(p[4], sg), bf16x2_mul(p[6], sg), bf16x2_mul(p[5], sg8),
-                          bf16x2_mul(p[7], sg8));
+          av[bb][0] = bf16x2_mul(p[0], sg);
+          av[bb][1] = bf16x2_mul(p[2], sg);
+          av[bb][2] = bf16x2_mul(p[1], sg8);
+          av[bb][3] = bf16x2_mul(p[3], sg8);
+          av[bb][4] = bf16x2_mul(p[4], sg);
+          av[bb][5] = bf16x2_mul(p[6], sg);
+          av[bb][6] = bf16x2_mul(p[5], sg8);
+          av[bb][7] = bf16x2_mul(p[7], sg8);
+        }
+        waitb(&B.aempty[sa], ((cnt / kAStages) & 1) ^ 1, B, a.status);
+        // The MMAs of chunk cnt - kAStages have completed (the commit that freed this A stage
+        // follows them): their shared-memory stage, whose codes this warp read long ago, is free.
+        if (cnt >= kAStages) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.empty[(cnt - kAStages) % kStages]);
+        }
+        tc_fence_after();
+        const uint32_t acol = tbase + lane_base + kTmemA0 + (sa * kMT + m) * 64;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          tmem_st_16x256b(acol + 16 * bb, av[bb][0], av[bb][1], av[bb][2], av[bb][3]);
+          tmem_st_16x256b(acol + 16 * bb + 8, av[bb][4], av[bb][5], av[bb][6], av[bb][7]);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -249,14 +276,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         tmem_wait_ld();
         const int nmax = min(32, ntok - col0);
         if (MODE == 0) {
+          // Lane rho < 8 holds gate row i of its unit, lane rho + 8 the up row of the same i.  For each
+          // pair of token columns (n, n + 1) the gate lane finishes column n and the up lane column n + 1.
           const int r = 32 * q + lane, tu = r >> 4, rho = r & 15;
+          const bool gate_lane = rho < 8;
           const int i = (mt * kTileUnits + tu) * 8 + (rho & 7);
           const int I = a.G.I;
 #pragma unroll
-          for (int n = 0; n < 32; ++n) {
-            const float up = __shfl_down_sync(0xffffffffu, __uint_as_float(v[n]), 8);
-            if (rho < 8 && n < nmax)
-              a.h_out[(size_t)(it.y + col0 + n) * I + i] = float_to_bf16_bits(silu_f(__uint_as_float(v[n])) * up);
+          for (int n = 0; n < 32; n += 2) {
+            const float mine0 = __uint_as_float(v[n]), mine1 = __uint_as_float(v[n + 1]);
+            const float other = __shfl_xor_sync(0xffffffffu, gate_lane ? mine1 : mine0, 8);
+            const float gv = gate_lane ? mine0 : other, uv = gate_lane ? other : mine1;
+            const int nn = gate_lane ? n : n + 1;
+            if (nn < nmax) a.h_out[(size_t)(it.y + col0 + nn) * I + i] = float_to_bf16_bits(silu_fast(gv) * uv);
           }
         } else {
           const int H = a.G.H;
