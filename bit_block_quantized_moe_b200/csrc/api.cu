@@ -58,6 +58,10 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const bool fused = decode_fused_supported(d, T);
   const size_t o_tcnt = take(fused ? decode_counter_words(d) * 4 : 0);
   const size_t o_part = take(fused ? decode_partial_floats(d, T) * 4 : 0);
+  const bool rtc = router_tc_supported(d, T);
+  const int rks = rtc ? router_tc_ksplit(d, T) : 1;
+  const size_t o_wsplit = take(rtc ? (size_t)3 * E * H * 2 : 0);
+  const size_t o_rpart = take(rks > 1 ? (size_t)rks * T * E * 4 : 0);
   if (base && ws) {
     uint8_t *b = static_cast<uint8_t *>(base);
     ws->status = reinterpret_cast<uint32_t *>(b + o_hdr);
@@ -84,6 +88,8 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->gbar = reinterpret_cast<uint64_t *>(b + o_hdr + 64);
     ws->tile_cnt = reinterpret_cast<uint32_t *>(b + o_tcnt);
     ws->partial = reinterpret_cast<float *>(b + o_part);
+    ws->wsplit = rtc ? reinterpret_cast<uint16_t *>(b + o_wsplit) : nullptr;
+    ws->rpart = reinterpret_cast<float *>(b + o_rpart);
     ws->words = (int)words;
     ws->max_items = max_items;
   }

@@ -30,6 +30,8 @@ struct Workspace {
   uint64_t *gbar;          // grid barrier of the fused decode kernel: monotonic arrival counter
   uint32_t *tile_cnt;      // fused decode: per-tile arrival counters, then per-expert ready counters
   float *partial;          // fused decode: per (expert, tile) partial outputs
+  uint16_t *wsplit;        // tcgen05 router: [3][E][H] bf16 planes of the router weights (null: legacy router)
+  float *rpart;            // tcgen05 router: [ksplit][T][E] K-split partial logits (ksplit > 1)
   int words;               // ceil(T / 32)
   int max_items;
   int max_tc_items;
@@ -57,6 +59,10 @@ size_t decode_counter_words(const moe_dims &d);
 cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias,
                                 const uint8_t *experts, const uint8_t *shared, int T, const Workspace &ws,
                                 int32_t *idx_out, float *w_out, uint16_t *out, cudaStream_t s);
+bool router_tc_supported(const moe_dims &d, int T);
+int router_tc_ksplit(const moe_dims &d, int T);
+cudaError_t launch_router_tc(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias, int T,
+                             const Workspace &ws, cudaStream_t s);
 cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,
                                     cudaStream_t s);
 

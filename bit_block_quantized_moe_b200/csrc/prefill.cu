@@ -28,8 +28,6 @@
 // The issuing thread of the MMAs is the pipeline's pace: everything it waits
 // on is taken off its path.  Accumulators are double-buffered so the epilogue
 // of one item overlaps the MMAs of the next.  Every wait is bounded (sync.cuh).
-#include <cudaTypedefs.h>
-
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -324,36 +322,11 @@ __global__ void gather_rows_kernel(const uint16_t *__restrict__ x, const int32_t
   for (int i = lane; i < H / 8; i += 32) dst[i] = src[i];
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2-D map over a row-major bf16 matrix [rows][cols], boxes of box_rows x 64 columns, 128-byte swizzle.
-bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols, int box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // 4-D map over packed units: (32-bit word within a 640-byte block group, group, unit, expert);
 // one box is one group of 16 consecutive units (10240 bytes, no swizzle).
 bool make_units_map(CUtensorMap *map, const void *base, int groups, int units, int experts, size_t unit_bytes,
                     size_t expert_bytes) {
-  auto fn = encode_fn();
+  auto fn = tma_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {kGroupBytes / 4, (cuuint64_t)groups, (cuuint64_t)units, (cuuint64_t)experts};
   const cuuint64_t strides[3] = {kGroupBytes, unit_bytes, expert_bytes};
@@ -378,6 +351,30 @@ bool make_maps(TcMaps *m, const uint8_t *experts, const uint8_t *shared, const P
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols, int box_rows) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t tc_smem_bytes() { return (size_t)kStages * kStageBytes + sizeof(Bars) + 1024; }
 

@@ -116,10 +116,6 @@ cudaError_t launch_pack(const uint8_t *canon, uint8_t *packed, int n_experts, co
 // Router logits, fp32 accumulation.  Also clears the dispatch bit map for this
 // call (stream order puts the clear before the top-k kernel's atomics).
 
-__device__ __forceinline__ void clear_range(uint32_t *p, size_t n) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
-}
-
 // Few tokens (T <= 8): one CTA of 2 warps per expert row, warp h summing the
 // row's half h (router_part), combined in half order.
 __global__ void __launch_bounds__(64) router_logits_small_kernel(const uint16_t *__restrict__ x,
@@ -141,20 +137,12 @@ __global__ void __launch_bounds__(64) router_logits_small_kernel(const uint16_t 
   if (threadIdx.x < T) logits[(size_t)threadIdx.x * E + e] = router_combine(part[threadIdx.x], bias ? bias[e] : 0.f);
 }
 
-// Many tokens: tensor cores with an exact 3-way bf16 split of the fp32 router
-// weights.  w = hi + mid + lo exactly (each a bf16 holding the next 8
-// significant bits); x is bf16 already, so every product is exact in fp32 and
-// only the fp32 accumulation rounds, as in a CUDA-core dot product.  Each
-// 256-wide K slice is accumulated in a fresh tensor-core accumulator and then
-// added to the running fp32 sum.
-__device__ __forceinline__ void split3_bf16(float w, uint16_t &hi, uint16_t &mid, uint16_t &lo) {
-  hi = float_to_bf16_bits(w);
-  const float r1 = w - bf16_bits_to_float(hi);
-  mid = float_to_bf16_bits(r1);
-  const float r2 = r1 - bf16_bits_to_float(mid);
-  lo = float_to_bf16_bits(r2);
-}
-
+// Many tokens without a split-weight workspace (the no-allocation routing
+// entry point) or with a hidden size that is not a multiple of 256: legacy
+// warp MMAs on the exact 3-way bf16 split of the fp32 router weights, split
+// in registers (split3_bf16).  Each 256-wide K slice is accumulated in a fresh
+// accumulator and then added to the running fp32 sum.  With a workspace the
+// tcgen05 router (router_tc.cu) is used instead.
 constexpr int kRbE = 64, kRbT = 32, kRbK = 64, kRbStages = 3;  // CTA tile: experts x tokens x K step
 constexpr int kRwStride = kRbK + 8;                                // floats (bank spread for float2 reads)
 constexpr int kRxStride = kRbK + 8;                                // bf16
@@ -289,6 +277,9 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, 
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, false, s);
     router_logits_small_kernel<<<E, 32 * kRouterParts, 0, s>>>(x, Wr, bias, T, H, E, ws.logits, ws.zero_begin, ws.zero_words);
     trace_mark(MOE_KERNEL_ROUTER_LOGITS, true, s);
+  } else if (ws.wsplit && router_tc_supported(d, T)) {
+    const cudaError_t e0 = launch_router_tc(d, x, Wr, bias, T, ws, s);
+    if (e0 != cudaSuccess) return e0;
   } else {
     dim3 grid((E + kRbE - 1) / kRbE, (T + kRbT - 1) / kRbT);
     cudaError_t e0 = cudaFuncSetAttribute(router_logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -45,6 +45,24 @@ __device__ __forceinline__ void router_part(const uint16_t *x, int xstride, int 
 
 __device__ __forceinline__ float router_combine(const float *parts, float b) { return (parts[0] + parts[1]) + b; }
 
+// Grid-stride clear of n words (the routing step's first kernel clears the
+// dispatch bit map and counters of the call).
+__device__ __forceinline__ void clear_range(uint32_t *p, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
+}
+
+// Exact 3-way bf16 split of an fp32 router weight: w = hi + mid + lo, each a
+// bf16 holding the next 8 significant bits of the remainder.  With bf16
+// tokens every product token * part is exact in fp32, so a tensor-core dot
+// product over the three parts rounds only in its fp32 accumulation.
+__device__ __forceinline__ void split3_bf16(float w, uint16_t &hi, uint16_t &mid, uint16_t &lo) {
+  hi = float_to_bf16_bits(w);
+  const float r1 = w - bf16_bits_to_float(hi);
+  mid = float_to_bf16_bits(r1);
+  const float r2 = r1 - bf16_bits_to_float(mid);
+  lo = float_to_bf16_bits(r2);
+}
+
 // fp32 softmax over the k winners held by lanes 0..k-1 (lane order = selection order).
 __device__ __forceinline__ float topk_softmax(float myv, int lane, int k) {
   const float mx = __shfl_sync(0xffffffffu, myv, 0);

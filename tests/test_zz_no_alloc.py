@@ -1,13 +1,19 @@
 """moe_route_noalloc: routing for callers that cannot allocate device memory
 (inside a stream capture, under a pre-reserved memory pool, or in loops that
 cannot afford an allocation's device synchronisation).  Its scratch is a static
-device array inside the library; this checks it against moe_route, which uses a
-caller-provided workspace, on two calls in a row.  Collected last on purpose."""
+device array inside the library; this checks it and moe_route, which uses a
+caller-provided workspace, against the oracle on two calls in a row.  With more
+than 8 tokens the two entry points use different router kernels (the workspace
+one holds the split router weights for the tcgen05 router), so their routing is
+only required to agree with the oracle's up to near-ties.  Collected last on
+purpose."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from gen import CONFIGS, make_router, make_x
+from parity import check_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -32,8 +38,12 @@ def test_noalloc_route_matches_workspace_route():
         M.moe_route(dims, x, Wd, bd, T, idx_a, w_a, ws)
         M.moe_route_noalloc(dims, x, Wd, bd, T, idx_b, w_b)
         torch.cuda.synchronize()
-        assert torch.equal(idx_a, idx_b), f"call {call}: expert sets differ"
-        assert torch.max(torch.abs(w_a - w_b)).item() <= 1e-5, f"call {call}: weights differ"
+        x_np = x.cpu().numpy().view(np.uint16)
+        idx_o, w_o, gap, _ = oracle.route(x_np, Wr, b, cfg.top_k)
+        check_routing(idx_a.cpu().numpy(), w_a.cpu().numpy(), idx_o, w_o, gap)
+        check_routing(idx_b.cpu().numpy(), w_b.cpu().numpy(), idx_o, w_o, gap)
+        if T <= 8:  # same router kernel on both sides: identical results
+            assert torch.equal(idx_a, idx_b) and torch.equal(w_a, w_b), f"call {call}: results differ"
 
     # sizes beyond the static scratch are rejected before any launch
     T_big = 262144 // cfg.n_experts + 1
