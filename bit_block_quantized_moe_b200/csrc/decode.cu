@@ -78,6 +78,12 @@ struct SmemLayout {
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
+// Warps that share one token's top-k selection (at most 4, and all T tokens' warps at once).
+__host__ __device__ inline int topk_warps_per_token(int T) {
+  const int w = kConsumerWarps / T;
+  return w < 1 ? 1 : (w > 4 ? 4 : w);
+}
+
 __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes) {
   SmemLayout L;
   uint32_t o = 0;
@@ -90,8 +96,8 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   L.rpart = o;  // [rows per pass][8 tokens][router parts]
   o += (kConsumerWarps / kRouterParts) * kMaxTok * kRouterParts * 4;
   o = align_to(o, 16);
-  L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
-  o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
+  L.red = o;  // top-k scratch (phase B: 64 uint64 per warp), then the h staging of phase D: [2][T][I + 16] bf16
+  o += align_to(max((uint32_t)kConsumerWarps * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
   L.sel_idx = o;
   o += kMaxSel * 4;
   L.sel_w = o;
@@ -244,9 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   {
     if (blockIdx.x == 0)
       for (int i = tid; i < G.dn_units + kMaxEntries; i += kConsumers) a.tile_cnt[i] = 0u;
+    constexpr int kRowsPerPass = kConsumerWarps / kRouterParts;  // one warp per router row part
+    // the bias of the logit this thread finishes in the first pass, loaded while the copies land
+    float bias0 = 0.f;
+    if (a.bias && tid < kRowsPerPass * T && tid / T < n_rrows) bias0 = __ldg(a.bias + blockIdx.x + gridDim.x * (tid / T));
     cp_async_wait_group<0>();  // this thread's pieces of the tokens and router rows have landed
     named_bar(kBarConsumers, kConsumers);
-    constexpr int kRowsPerPass = kConsumerWarps / kRouterParts;  // one warp per router row part
     for (int r0 = 0; r0 < n_rrows; r0 += kRowsPerPass) {
       const int r = r0 + warp / kRouterParts, q = warp % kRouterParts;
       if (r < n_rrows) {
@@ -262,17 +271,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         const int rr = tid / T, t = tid % T;
         if (r0 + rr < n_rrows) {
           const int e = blockIdx.x + gridDim.x * (r0 + rr);
-          a.logits[(size_t)t * E + e] =
-              router_combine(rpart + (rr * kMaxTok + t) * kRouterParts, a.bias ? a.bias[e] : 0.f);
+          a.logits[(size_t)t * E + e] = router_combine(rpart + (rr * kMaxTok + t) * kRouterParts,
+                                                       r0 == 0 ? bias0 : (a.bias ? a.bias[e] : 0.f));
         }
       }
       named_bar(kBarConsumers, kConsumers);
     }
     // Arrive on the grid barrier, prepare the token rows as the B operand while the other CTAs finish
     // their logits (the router is done with them), then wait.
-    const uint64_t bar_target = grid_arrive(a.gbar, kBarConsumers, kConsumers, tid == 0);
+    // The barrier's leader is the last thread, which has the fewest token-row pieces to prepare, so
+    // that its fence and atomic round trip overlap the others' preparation.
+    const bool leader = tid == kConsumers - 1;
+    const uint64_t bar_target = grid_arrive(a.gbar, kBarConsumers, kConsumers, leader);
     prep_rows(xs, xstride, H, T, corr, tid);
-    grid_wait(a.gbar, bar_target, kBarConsumers, kConsumers, tid == 0, a.status, &misc[2]);
+    grid_wait(a.gbar, bar_target, kBarConsumers, kConsumers, leader, a.status, &misc[2]);
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
     // All logits into shared memory first (one coalesced pass through L2), then one warp per token.
@@ -281,14 +293,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       reinterpret_cast<float4 *>(lg)[i] = ldg_cg_f4(a.logits + 4 * (size_t)i);
     for (int i = (T * E / 4) * 4 + tid; i < T * E; i += kConsumers) lg[i] = __ldcg(a.logits + i);
     named_bar(kBarConsumers, kConsumers);
+    // W warps per token: each selects the top-k of a slice of the token's logits, then one warp merges
+    // the W * k candidates by rank.  The selection key (logit desc, index asc) and the softmax are
+    // those of the one-warp selection, so the result is the same.
+    const int W = topk_warps_per_token(T);
+    int e = 0;
+    float wt = 0.f;
+    uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
+    if (W == 1) {
+      if (warp < T) {
+        if (E <= 512)
+          warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+        else
+          warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+      }
+    } else {
+      const int cstride = (W * K + 1) & ~1;  // keeps every token's candidates 16-byte aligned
+      uint64_t *cand = reinterpret_cast<uint64_t *>(ring + align_to((uint32_t)T * E * 4, 16));
+      const int slice = (E + W - 1) / W;
+      if (warp < T * W) {
+        const int t = warp / W, part = warp % W;
+        const int lo = min(E, part * slice), n = min(E, lo + slice) - lo;
+        const float *row = lg + (size_t)t * E + lo;
+        uint64_t key;
+        if (slice <= 128)
+          key = warp_topk_key<4, true>(row, n, lo, K, lane, scratch);
+        else if (slice <= 256)
+          key = warp_topk_key<8, true>(row, n, lo, K, lane, scratch);
+        else
+          key = warp_topk_key<16, true>(row, n, lo, K, lane, scratch);
+        if (lane < K) cand[t * cstride + part * K + lane] = key;
+      }
+      named_bar(kBarConsumers, kConsumers);
+      if (warp < T) {
+        const uint64_t mine = warp_merge_keys(cand + (size_t)warp * cstride, W * K, K, lane, scratch);
+        e = (int)~(uint32_t)mine;
+        wt = topk_softmax(key_float((uint32_t)(mine >> 32)), lane, K);
+      }
+    }
     if (warp < T) {
-      int e;
-      float wt;
-      uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
-      if (E <= 512)
-        warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
-      else
-        warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
       if (lane < K) {
         sel_idx[warp * K + lane] = e;
         sel_w[warp * K + lane] = wt;
@@ -586,7 +629,10 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   if ((max_entries * G.dn_units + n_sm - 1) / n_sm > kMaxSel) return cudaErrorInvalidConfiguration;
   const int rrows = (d.n_experts + n_sm - 1) / n_sm;  // router rows per CTA, staged in the ring
   if ((size_t)rrows * d.hidden * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;
-  if ((size_t)T * d.n_experts * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;  // logits
+  // logits, then the top-k candidates of the split selection
+  const size_t cand_bytes = (size_t)T * ((topk_warps_per_token(T) * d.top_k + 1) & ~1) * 8;
+  if (align_to((uint32_t)(T * d.n_experts * 4), 16) + cand_bytes > (size_t)ns * stage_bytes)
+    return cudaErrorInvalidConfiguration;
 
   DecodeArgs a{};
   a.x = x;

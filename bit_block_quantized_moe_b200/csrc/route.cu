@@ -7,6 +7,8 @@
 // selected set and the bias placement are this library's stated readings.
 #include <float.h>
 
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "router.cuh"
 #include "sync.cuh"
@@ -326,7 +328,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int &
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int ws = warp_sums[lane];
+    int ws = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
     int wi = ws;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -343,58 +345,31 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int &
   return r;
 }
 
-__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(const uint32_t *__restrict__ bitmap, int words,
-                                                                     int E, int T, int k,
-                                                                     uint32_t *__restrict__ wprefix, int32_t *counts,
+// Per expert (one CTA each): exclusive popcount prefix of its membership words
+// and its token count.
+__global__ void __launch_bounds__(kScanThreads) dispatch_wscan_kernel(const uint32_t *__restrict__ bitmap, int words,
+                                                                      uint32_t *__restrict__ wprefix,
+                                                                      int32_t *__restrict__ counts) {
+  __shared__ int warp_sums[33];
+  const int e = blockIdx.x;
+  int run = 0;
+  for (int w0 = 0; w0 < words; w0 += blockDim.x) {
+    const int wi = w0 + threadIdx.x;
+    const uint32_t bits = wi < words ? bitmap[(size_t)e * words + wi] : 0u;
+    int tot;
+    const int ex = block_exclusive_scan(__popc(bits), warp_sums, tot);
+    if (wi < words) wprefix[(size_t)e * words + wi] = (uint32_t)(run + ex);
+    run += tot;
+  }
+  if (threadIdx.x == 0) counts[e] = run;
+}
+
+// Expert offsets and the work lists from the per-expert counts (one CTA).
+__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int T, int k,
+                                                                     const int32_t *__restrict__ counts,
                                                                      int32_t *offsets, int4 *items, uint32_t *n_items,
                                                                      int4 *tc_items, uint32_t *n_tc_items) {
   __shared__ int warp_sums[33];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kNW = kScanThreads / 32;
-  if (words <= 32) {
-    // one word per lane: load 8 experts' words at once so their L2 round trips overlap
-    for (int e0 = warp; e0 < E; e0 += 8 * kNW) {
-      uint32_t bits[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = e0 + j * kNW;
-        bits[j] = (e < E && lane < words) ? bitmap[(size_t)e * words + lane] : 0u;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = e0 + j * kNW;
-        const uint32_t cnt = __popc(bits[j]);
-        uint32_t incl = cnt;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += v;
-        }
-        if (e < E) {
-          if (lane < words) wprefix[(size_t)e * words + lane] = incl - cnt;
-          if (lane == 31) counts[e] = (int32_t)incl;
-        }
-      }
-    }
-  } else
-  for (int e = warp; e < E; e += kNW) {
-    uint32_t run = 0;
-    for (int w0 = 0; w0 < words; w0 += 32) {
-      const int wi = w0 + lane;
-      const uint32_t bits = wi < words ? bitmap[(size_t)e * words + wi] : 0u;
-      const uint32_t cnt = __popc(bits);
-      uint32_t incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      if (wi < words) wprefix[(size_t)e * words + wi] = run + incl - cnt;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) counts[e] = (int32_t)run;
-  }
-  __syncthreads();
   // thread i owns experts [i * per, (i + 1) * per)
   const int per = (E + kScanThreads - 1) / kScanThreads;
   const int eb = threadIdx.x * per, ee = min(E, eb + per);
@@ -416,14 +391,15 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(const uint3
     for (int j = 0; j < c; j += 64) tc_items[itc++] = make_int4(i, pos + j, min(64, c - j), 0);
     pos += c;
   }
+  // the shared expert's items follow the routed ones
+  const int shared_items = (T + 7) >> 3, shared_tc = (T + 63) >> 6;
+  for (int i = threadIdx.x; i < shared_items; i += blockDim.x)
+    items[tot_items + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
+  for (int i = threadIdx.x; i < shared_tc; i += blockDim.x)
+    tc_items[tot_tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
   if (threadIdx.x == 0) {
     offsets[E] = tot_cnt;  // == T * k when every index was valid
-    const int shared_items = (T + 7) >> 3;
-    for (int i = 0; i < shared_items; ++i) items[tot_items + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
     *n_items = (uint32_t)(tot_items + shared_items);
-    const int shared_tc = (T + 63) >> 6;
-    for (int i = 0; i < shared_tc; ++i)
-      tc_items[tot_tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
     *n_tc_items = (uint32_t)(tot_tc + shared_tc);
   }
 }
@@ -483,8 +459,10 @@ cudaError_t launch_dispatch_bits(const moe_dims &d, int T, const Workspace &ws, 
 cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s) {
   const int E = d.n_experts, k = d.top_k;
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, false, s);
-  dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(ws.bitmap, ws.words, E, T, k, ws.wprefix, ws.counts, ws.offsets,
-                                                  ws.items, ws.n_items, ws.tc_items, ws.n_tc_items);
+  const int wthreads = std::min(kScanThreads, (ws.words + 31) & ~31);
+  dispatch_wscan_kernel<<<E, wthreads, 0, s>>>(ws.bitmap, ws.words, ws.wprefix, ws.counts);
+  dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(E, T, k, ws.counts, ws.offsets, ws.items, ws.n_items, ws.tc_items,
+                                                  ws.n_tc_items);
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, true, s);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
