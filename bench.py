@@ -56,7 +56,8 @@ def parse():
 
 # Sources the fused decode kernel is compiled from; an ncu summary under profiles/ records
 # their hash, and its DRAM traffic is reported only while the sources still match.
-DECODE_SOURCES = ["decode.cu", "common.cuh", "sync.cuh", "router.cuh", "kernels.cuh"]
+# the files that make up the fused decode kernel's device code (kernels.cuh holds host declarations only)
+DECODE_SOURCES = ["decode.cu", "common.cuh", "sync.cuh", "router.cuh"]
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_fused_kernel_t3.md")
 
 
