@@ -50,7 +50,8 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_sw = take(slots * 4);
   const int max_items = max_items_for(d, T, 8);
   const size_t o_items = take((size_t)max_items * 16);
-  const int max_tc_items = max_items_for(d, T, 64);
+  const int tc_n = tc_item_tokens(d, T);
+  const int max_tc_items = max_items_for(d, T, tc_n);
   const size_t o_tc_items = take((size_t)max_tc_items * 16);
   const size_t o_xs = take(T > 8 ? slots * H * 2 : 0);
   const size_t o_h = take(slots * I * 2);
@@ -83,6 +84,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->n_tc_items = reinterpret_cast<uint32_t *>(b + o_hdr + 8);
     ws->xs = reinterpret_cast<uint16_t *>(b + o_xs);
     ws->max_tc_items = max_tc_items;
+    ws->tc_item_tokens = tc_n;
     ws->h = reinterpret_cast<uint16_t *>(b + o_h);
     ws->y = reinterpret_cast<float *>(b + o_y);
     ws->gbar = reinterpret_cast<uint64_t *>(b + o_hdr + 64);

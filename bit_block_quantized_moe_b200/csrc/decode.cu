@@ -78,12 +78,6 @@ struct SmemLayout {
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Warps that share one token's top-k selection (at most 4, and all T tokens' warps at once).
-__host__ __device__ inline int topk_warps_per_token(int T) {
-  const int w = kConsumerWarps / T;
-  return w < 1 ? 1 : (w > 4 ? 4 : w);
-}
-
 __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes) {
   SmemLayout L;
   uint32_t o = 0;
@@ -96,8 +90,8 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   L.rpart = o;  // [rows per pass][8 tokens][router parts]
   o += (kConsumerWarps / kRouterParts) * kMaxTok * kRouterParts * 4;
   o = align_to(o, 16);
-  L.red = o;  // top-k scratch (phase B: 64 uint64 per warp), then the h staging of phase D: [2][T][I + 16] bf16
-  o += align_to(max((uint32_t)kConsumerWarps * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
+  L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
+  o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
   L.sel_idx = o;
   o += kMaxSel * 4;
   L.sel_w = o;
@@ -293,45 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       reinterpret_cast<float4 *>(lg)[i] = ldg_cg_f4(a.logits + 4 * (size_t)i);
     for (int i = (T * E / 4) * 4 + tid; i < T * E; i += kConsumers) lg[i] = __ldcg(a.logits + i);
     named_bar(kBarConsumers, kConsumers);
-    // W warps per token: each selects the top-k of a slice of the token's logits, then one warp merges
-    // the W * k candidates by rank.  The selection key (logit desc, index asc) and the softmax are
-    // those of the one-warp selection, so the result is the same.
-    const int W = topk_warps_per_token(T);
-    int e = 0;
-    float wt = 0.f;
-    uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
-    if (W == 1) {
-      if (warp < T) {
-        if (E <= 512)
-          warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
-        else
-          warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
-      }
-    } else {
-      const int cstride = (W * K + 1) & ~1;  // keeps every token's candidates 16-byte aligned
-      uint64_t *cand = reinterpret_cast<uint64_t *>(ring + align_to((uint32_t)T * E * 4, 16));
-      const int slice = (E + W - 1) / W;
-      if (warp < T * W) {
-        const int t = warp / W, part = warp % W;
-        const int lo = min(E, part * slice), n = min(E, lo + slice) - lo;
-        const float *row = lg + (size_t)t * E + lo;
-        uint64_t key;
-        if (slice <= 128)
-          key = warp_topk_key<4, true>(row, n, lo, K, lane, scratch);
-        else if (slice <= 256)
-          key = warp_topk_key<8, true>(row, n, lo, K, lane, scratch);
-        else
-          key = warp_topk_key<16, true>(row, n, lo, K, lane, scratch);
-        if (lane < K) cand[t * cstride + part * K + lane] = key;
-      }
-      named_bar(kBarConsumers, kConsumers);
-      if (warp < T) {
-        const uint64_t mine = warp_merge_keys(cand + (size_t)warp * cstride, W * K, K, lane, scratch);
-        e = (int)~(uint32_t)mine;
-        wt = topk_softmax(key_float((uint32_t)(mine >> 32)), lane, K);
-      }
-    }
     if (warp < T) {
+      int e;
+      float wt;
+      uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
+      if (E <= 512)
+        warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+      else
+        warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
       if (lane < K) {
         sel_idx[warp * K + lane] = e;
         sel_w[warp * K + lane] = wt;
@@ -629,10 +592,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   if ((max_entries * G.dn_units + n_sm - 1) / n_sm > kMaxSel) return cudaErrorInvalidConfiguration;
   const int rrows = (d.n_experts + n_sm - 1) / n_sm;  // router rows per CTA, staged in the ring
   if ((size_t)rrows * d.hidden * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;
-  // logits, then the top-k candidates of the split selection
-  const size_t cand_bytes = (size_t)T * ((topk_warps_per_token(T) * d.top_k + 1) & ~1) * 8;
-  if (align_to((uint32_t)(T * d.n_experts * 4), 16) + cand_bytes > (size_t)ns * stage_bytes)
-    return cudaErrorInvalidConfiguration;
+  if ((size_t)T * d.n_experts * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;  // logits
 
   DecodeArgs a{};
   a.x = x;

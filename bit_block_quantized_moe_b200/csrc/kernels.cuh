@@ -22,7 +22,7 @@ struct Workspace {
   int32_t *sorted_tok;     // [T*k + T]: token of each sorted position (shared slots last)
   float *sorted_w;         // [T*k + T]
   int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)
-  int4 *tc_items;          // [max_tc_items]: (expert, first position, tokens <= 64, 0)
+  int4 *tc_items;          // [max_tc_items]: (expert, first position, tokens <= tc_item_tokens, 0)
   uint32_t *n_tc_items;
   uint16_t *xs;            // [T*k + T][H] bf16 token rows in sorted-position order
   uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position
@@ -35,6 +35,7 @@ struct Workspace {
   int words;               // ceil(T / 32)
   int max_items;
   int max_tc_items;
+  int tc_item_tokens;       // 64 or 128 (tc_item_tokens())
 };
 
 // Profiling hook (moe_trace_kernel): records the caller's events around kernel `id`.
@@ -50,6 +51,8 @@ cudaError_t launch_dispatch_bits(const moe_dims &d, int T, const Workspace &ws, 
 cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                            const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
+// Tokens per tcgen05 prefill work item for T tokens (64, or 128 once an expert averages 64 tokens).
+int tc_item_tokens(const moe_dims &d, int T);
 cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                               const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s);

@@ -2,21 +2,23 @@
 // (tcgen05, sm_100a).
 //
 // One persistent CTA per SM walks a list of work items (expert, two 128-row
-// M tiles, up to 64 tokens): the two tiles share every load of the expert's
+// M tiles, up to 64 tokens; or, once experts average 64 tokens, one M tile and
+// up to 128 tokens): the tiles of an item share every load of the expert's
 // token rows.  For each 128-wide K chunk:
-//   producer warp    : one TMA load of both tiles' packed Q2 codes + scales
-//                      (16 units x 640 B, a 4-D tensor map over the experts;
-//                      units past the expert's last tile read as zeros) and
-//                      two of the expert's token rows (slot-sorted
-//                      activations, 128-byte swizzle, 16/32/64-row boxes)
-//                      into one of 8 shared-memory stages;
+//   producer warp    : one TMA load of the tiles' packed Q2 codes + scales
+//                      (8 units x 640 B per tile, a 4-D tensor map over the
+//                      experts; units past the expert's last tile read as
+//                      zeros) and two of the expert's token rows (slot-sorted
+//                      activations, 128-byte swizzle, 16/32/64/128-row boxes)
+//                      into one of 8 (5) shared-memory stages;
 //   16 dequant warps : decode the codes in registers to bf16 d * (q - 1)
 //                      while the tensor core still reads the A stage they
 //                      will fill, then store them (tcgen05.st), one 16-row
-//                      unit (4 blocks) per warp; once the MMAs of a chunk
+//                      unit (4 blocks) per warp (half a unit with one M
+//                      tile); once the MMAs of a chunk
 //                      have completed they also release its shared-memory
 //                      stage to the producer;
-//   MMA warp        : 2 x 8 tcgen05.mma per chunk (A from tensor memory, B
+//   MMA warp        : 8 tcgen05.mma per M tile and chunk (A from tensor memory, B
 //                     from shared memory), fp32 accumulators in tensor
 //                     memory, one commit per chunk.  It waits only on the A
 //                     stage: the dequant warps passed the chunk's TMA barrier
@@ -35,28 +37,40 @@ namespace moe {
 
 namespace {
 
-constexpr int kMT = 2;             // 128-row M tiles per work item: they share every token-row load
-constexpr int kStages = 8;         // shared-memory stages (A codes + B rows)
-constexpr int kAStages = 2;        // tensor-memory A stages (kMT x 64 columns each)
 constexpr int kTileUnits = 8;      // 16-row units per 128-row M tile
-constexpr int kMaxN = 64;          // tokens per work item
-constexpr int kABytes = kMT * kTileUnits * kGroupBytes;  // 10240
-constexpr int kBSub = kMaxN * 128;                       // one 64-wide K half of the chunk: 8 KB
-constexpr int kStageBytes = kABytes + 2 * kBSub;         // 26624 (a multiple of 1024)
 constexpr int kWarpProducer = 0, kWarpMMA = 1, kWarpDequant0 = 2, kNumDequant = 16, kWarpEpi0 = 18, kNumEpi = 4;
 constexpr int kThreadsTC = (kWarpEpi0 + kNumEpi) * 32;  // 704
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kDCols = kMT * kMaxN;      // one accumulator buffer: kMT M tiles x 64 token columns
-constexpr uint32_t kTmemA0 = 2 * kDCols;      // D buffers at columns 0 and kDCols; A stages from 256
-static_assert(kTmemA0 + kAStages * kMT * 64 <= kTmemCols, "tensor memory columns");
-static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment for the 128-byte swizzle");
+
+// Two shapes of work item.  Few tokens per expert (the 1024-token chunk: about 20): two 128-row M tiles and
+// at most 64 tokens, so that both tiles share every token-row load.  Many tokens per expert: one M tile and
+// at most 128 tokens, so that each expert's codes are decoded half as often and every MMA covers twice the
+// tokens for about the same issue cost.
+template <int MT, int MAXN>
+struct TcCfg {
+  static constexpr int kMT = MT;                                  // 128-row M tiles per work item
+  static constexpr int kMaxN = MAXN;                              // tokens per work item
+  static constexpr int kABytes = MT * kTileUnits * kGroupBytes;   // codes + scales of one K chunk
+  static constexpr int kBSub = MAXN * 128;                        // one 64-wide K half of the token rows
+  static constexpr int kStageBytes = kABytes + 2 * kBSub;
+  static constexpr int kStages = MT == 2 ? 8 : 5;                 // shared-memory stages (A codes + B rows)
+  static constexpr int kAStages = 2;                              // tensor-memory A stages (MT x 64 columns)
+  static constexpr uint32_t kDCols = MT * MAXN;                   // one accumulator buffer
+  static constexpr uint32_t kTmemA0 = 2 * kDCols;                 // D buffers at 0 and kDCols, A stages after
+  static constexpr int kBlocksPerWarp = MT == 2 ? 4 : 2;          // blocks of its unit each dequant warp decodes
+  static_assert(kTmemA0 + kAStages * MT * 64 <= kTmemCols, "tensor memory columns");
+  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment for the 128-byte swizzle");
+  static_assert(kNumDequant * kBlocksPerWarp == MT * kTileUnits * 4, "every block of a chunk decoded once");
+};
+using CfgFew = TcCfg<2, 64>;
+using CfgMany = TcCfg<1, 128>;
 
 struct TcArgs {
   const uint8_t *experts;
   const uint8_t *shared;
   PackedGeom G;
   int E;
-  const int4 *items;          // (expert or E for shared, first sorted position, tokens <= 64, 0)
+  const int4 *items;          // (expert or E for shared, first sorted position, tokens <= kMaxN, 0)
   const uint32_t *n_items;
   int mtiles;                 // 128-row tiles per expert for this projection
   int mgroups;                // ceil(mtiles / kMT): work items per token item
@@ -68,13 +82,15 @@ struct TcArgs {
   uint32_t *status;
 };
 
+template <class C>
 struct Bars {
-  uint64_t full[kStages], empty[kStages], afull[kAStages], aempty[kAStages], dfull[2], dempty[2], done;
+  uint64_t full[C::kStages], empty[C::kStages], afull[C::kAStages], aempty[C::kAStages], dfull[2], dempty[2], done;
   uint32_t tmem;
   int abort;
 };
 
-__device__ __forceinline__ bool waitb(uint64_t *bar, uint32_t parity, Bars &B, uint32_t *status) {
+template <class BarsT>
+__device__ __forceinline__ bool waitb(uint64_t *bar, uint32_t parity, BarsT &B, uint32_t *status) {
   if (mbar_try_wait(bar, parity)) return true;
   if (*reinterpret_cast<volatile int *>(&B.abort)) return false;
   if (!mbar_wait(bar, parity)) {
@@ -104,15 +120,18 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
 struct TcMaps {
   CUtensorMap a_routed;  // packed units of the routed experts, 4-D (u32 in unit group, group, unit, expert)
   CUtensorMap a_shared;  // the shared expert, same shape with one expert
-  CUtensorMap b[3];      // token rows [positions][K] bf16, boxes of 16 / 32 / 64 rows x 64 columns
+  CUtensorMap b[4];      // token rows [positions][K] bf16, boxes of 16 / 32 / 64 / 128 rows x 64 columns
 };
 
-template <int MODE>  // 0: gate/up + SwiGLU -> h (bf16); 1: down -> y (fp32)
+template <int MODE, class C>  // MODE 0: gate/up + SwiGLU -> h (bf16); 1: down -> y (fp32)
 __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_constant__ TcMaps maps, TcArgs a) {
+  constexpr int kMT = C::kMT, kMaxN = C::kMaxN, kABytes = C::kABytes, kBSub = C::kBSub;
+  constexpr int kStageBytes = C::kStageBytes, kStages = C::kStages, kAStages = C::kAStages;
+  constexpr uint32_t kDCols = C::kDCols, kTmemA0 = C::kTmemA0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned start (pointer arithmetic on the shared array keeps shared-memory addressing)
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  Bars &B = *reinterpret_cast<Bars *>(smem + kStages * kStageBytes);
+  Bars<C> &B = *reinterpret_cast<Bars<C> *>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = (int)*a.n_items;
   const int n_work = n_items * a.mgroups;
@@ -146,7 +165,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
         const int4 it = a.items[w / a.mgroups];
         const int mt0 = (w % a.mgroups) * kMT;
-        const int bsel = it.z <= 16 ? 0 : (it.z <= 32 ? 1 : 2);
+        const int bsel = it.z <= 16 ? 0 : (it.z <= 32 ? 1 : (it.z <= 64 ? 2 : 3));
         const int nrows = 16 << bsel;
         const CUtensorMap *amap = it.x == a.E ? &maps.a_shared : &maps.a_routed;
         const int ae = it.x == a.E ? 0 : it.x;
@@ -200,9 +219,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       if (!mbar_wait(&B.done, 0)) set_status(a.status, kStatusTimeout);
     }
   } else if (warp < kWarpEpi0) {
-    // ---- dequant warps: 4 per TMEM lane quadrant = kMT (2) M tiles x 2 units, one whole unit each ----
+    // ---- dequant warps: 4 per TMEM lane quadrant (the quadrant holds units 2q, 2q + 1 of each M tile):
+    // with two M tiles one whole unit each, with one tile half a unit (2 of its 4 blocks) each ----
     const int dw = warp - kWarpDequant0;
-    const int q = warp & 3, uq = (dw >> 2) & 1, m = dw >> 3;
+    const int q = warp & 3, uq = (dw >> 2) & 1;
+    const int m = kMT == 2 ? dw >> 3 : 0;
+    const int bb0 = kMT == 2 ? 0 : 2 * (dw >> 3);
+    constexpr int kNB = C::kBlocksPerWarp;
     const int unit = 2 * q + uq;
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * uq) << 16;
     const int g = lane >> 2;
@@ -218,13 +241,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
         // the whole unit in registers before the A stage is free: registers P0, P2 belong to row g,
         // P1, P3 to row g+8
-        uint32_t av[4][8];
+        uint32_t av[kNB][8];
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
+        for (int bb = 0; bb < kNB; ++bb) {
           uint32_t p[8];
-          decode_q2_exact(cws[bb], p);
+          const uint32_t cword = kNB == 4 ? cws[bb] : (bb0 == 0 ? cws[bb] : cws[2 + bb]);
+          const uint32_t sword = kNB == 4 ? sws[bb] : (bb0 == 0 ? sws[bb] : sws[2 + bb]);
+          decode_q2_exact(cword, p);
           uint32_t sg, sg8;
-          scale_pairs(sws[bb], sg, sg8);
+          scale_pairs(sword, sg, sg8);
           av[bb][0] = bf16x2_mul(p[0], sg);
           av[bb][1] = bf16x2_mul(p[2], sg);
           av[bb][2] = bf16x2_mul(p[1], sg8);
@@ -244,9 +269,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         tc_fence_after();
         const uint32_t acol = tbase + lane_base + kTmemA0 + (sa * kMT + m) * 64;
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          tmem_st_16x256b(acol + 16 * bb, av[bb][0], av[bb][1], av[bb][2], av[bb][3]);
-          tmem_st_16x256b(acol + 16 * bb + 8, av[bb][4], av[bb][5], av[bb][6], av[bb][7]);
+        for (int bb = 0; bb < kNB; ++bb) {
+          tmem_st_16x256b(acol + 16 * (bb0 + bb), av[bb][0], av[bb][1], av[bb][2], av[bb][3]);
+          tmem_st_16x256b(acol + 16 * (bb0 + bb) + 8, av[bb][4], av[bb][5], av[bb][6], av[bb][7]);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -323,14 +348,14 @@ __global__ void gather_rows_kernel(const uint16_t *__restrict__ x, const int32_t
 }
 
 // 4-D map over packed units: (32-bit word within a 640-byte block group, group, unit, expert);
-// one box is one group of 16 consecutive units (10240 bytes, no swizzle).
+// one box is one group of box_units consecutive units (640 bytes each, no swizzle).
 bool make_units_map(CUtensorMap *map, const void *base, int groups, int units, int experts, size_t unit_bytes,
-                    size_t expert_bytes) {
+                    size_t expert_bytes, int box_units) {
   auto fn = tma_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {kGroupBytes / 4, (cuuint64_t)groups, (cuuint64_t)units, (cuuint64_t)experts};
   const cuuint64_t strides[3] = {kGroupBytes, unit_bytes, expert_bytes};
-  const cuuint32_t box[4] = {kGroupBytes / 4, 1, kTileUnits * kMT, 1};
+  const cuuint32_t box[4] = {kGroupBytes / 4, 1, (cuuint32_t)box_units, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -338,15 +363,15 @@ bool make_units_map(CUtensorMap *map, const void *base, int groups, int units, i
 }
 
 bool make_maps(TcMaps *m, const uint8_t *experts, const uint8_t *shared, const PackedGeom &G, int E, bool down,
-               const void *rows, int P) {
+               const void *rows, int P, int mt) {
   const int groups = down ? G.dn_groups : G.gu_groups;
   const int units = down ? G.dn_units : G.gu_units;
   const size_t ub = down ? G.dn_unit_bytes : G.gu_unit_bytes;
   const size_t off = down ? G.gu_bytes : 0;
   const int K = down ? G.I : G.H;
-  bool ok = make_units_map(&m->a_routed, experts + off, groups, units, E, ub, G.expert_bytes) &&
-            make_units_map(&m->a_shared, shared + off, groups, units, 1, ub, G.expert_bytes);
-  for (int i = 0; i < 3 && ok; ++i) ok = make_rows_map(&m->b[i], rows, P, K, 16 << i);
+  bool ok = make_units_map(&m->a_routed, experts + off, groups, units, E, ub, G.expert_bytes, kTileUnits * mt) &&
+            make_units_map(&m->a_shared, shared + off, groups, units, 1, ub, G.expert_bytes, kTileUnits * mt);
+  for (int i = 0; i < 4 && ok; ++i) ok = make_rows_map(&m->b[i], rows, P, K, 16 << i);
   return ok;
 }
 
@@ -376,21 +401,20 @@ bool make_rows_map(CUtensorMap *map, const void *base, int rows, int cols, int b
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t tc_smem_bytes() { return (size_t)kStages * kStageBytes + sizeof(Bars) + 1024; }
+namespace {
 
-cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
-                              const uint16_t *x, int T, const Workspace &ws, cudaStream_t s) {
-  const int P = T * d.top_k + T;  // sorted positions (routed + shared)
-  trace_mark(MOE_KERNEL_GATHER, false, s);
-  gather_rows_kernel<<<(unsigned)(((long long)P * 32 + 255) / 256), 256, 0, s>>>(x, ws.sorted_tok, P, G.H, ws.xs);
-  trace_mark(MOE_KERNEL_GATHER, true, s);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+template <class C>
+size_t tc_smem_bytes() {
+  return (size_t)C::kStages * C::kStageBytes + sizeof(Bars<C>) + 1024;
+}
 
+template <class C>
+cudaError_t launch_tc_pair(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
+                           int P, const Workspace &ws, cudaStream_t s) {
   int dev = 0, n_sm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  const size_t smem = tc_smem_bytes();
+  const size_t smem = tc_smem_bytes<C>();
   TcArgs a{};
   a.experts = experts;
   a.shared = shared;
@@ -403,36 +427,56 @@ cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint
   a.y_out = ws.y;
 
   TcMaps maps_gu, maps_dn;
-  if (!make_maps(&maps_gu, experts, shared, G, d.n_experts, false, ws.xs, P) ||
-      !make_maps(&maps_dn, experts, shared, G, d.n_experts, true, ws.h, P))
+  if (!make_maps(&maps_gu, experts, shared, G, d.n_experts, false, ws.xs, P, C::kMT) ||
+      !make_maps(&maps_dn, experts, shared, G, d.n_experts, true, ws.h, P, C::kMT))
     return cudaErrorInvalidValue;
 
   // gate/up + SwiGLU: M = 2I interleaved rows (8 gate + 8 up per unit), K = H
   a.mtiles = G.gu_units / kTileUnits;
-  a.mgroups = (a.mtiles + kMT - 1) / kMT;
+  a.mgroups = (a.mtiles + C::kMT - 1) / C::kMT;
   a.kchunks = G.gu_groups;
   a.unit_bytes = G.gu_unit_bytes;
   a.sec_off = 0;
-  err = cudaFuncSetAttribute(tc_expert_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = cudaFuncSetAttribute(tc_expert_kernel<0, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   trace_mark(MOE_KERNEL_GATE_UP, false, s);
-  tc_expert_kernel<0><<<n_sm, kThreadsTC, smem, s>>>(maps_gu, a);
+  tc_expert_kernel<0, C><<<n_sm, kThreadsTC, smem, s>>>(maps_gu, a);
   trace_mark(MOE_KERNEL_GATE_UP, true, s);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
 
   // down: M = H rows, K = I
   a.mtiles = G.dn_units / kTileUnits;
-  a.mgroups = (a.mtiles + kMT - 1) / kMT;
+  a.mgroups = (a.mtiles + C::kMT - 1) / C::kMT;
   a.kchunks = G.dn_groups;
   a.unit_bytes = G.dn_unit_bytes;
   a.sec_off = G.gu_bytes;
-  err = cudaFuncSetAttribute(tc_expert_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  err = cudaFuncSetAttribute(tc_expert_kernel<1, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   trace_mark(MOE_KERNEL_DOWN, false, s);
-  tc_expert_kernel<1><<<n_sm, kThreadsTC, smem, s>>>(maps_dn, a);
+  tc_expert_kernel<1, C><<<n_sm, kThreadsTC, smem, s>>>(maps_dn, a);
   trace_mark(MOE_KERNEL_DOWN, true, s);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+int tc_item_tokens(const moe_dims &d, int T) {
+  // one M tile and 128-token items once an expert averages at least 64 tokens
+  return (long long)T * d.top_k >= 64LL * d.n_experts ? CfgMany::kMaxN : CfgFew::kMaxN;
+}
+
+cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
+                              const uint16_t *x, int T, const Workspace &ws, cudaStream_t s) {
+  const int P = T * d.top_k + T;  // sorted positions (routed + shared)
+  trace_mark(MOE_KERNEL_GATHER, false, s);
+  gather_rows_kernel<<<(unsigned)(((long long)P * 32 + 255) / 256), 256, 0, s>>>(x, ws.sorted_tok, P, G.H, ws.xs);
+  trace_mark(MOE_KERNEL_GATHER, true, s);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+
+  return tc_item_tokens(d, T) == CfgMany::kMaxN ? launch_tc_pair<CfgMany>(d, G, experts, shared, P, ws, s)
+                                                : launch_tc_pair<CfgFew>(d, G, experts, shared, P, ws, s);
 }
 
 }  // namespace moe

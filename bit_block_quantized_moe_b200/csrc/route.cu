@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_wscan_kernel(const uint
 __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int T, int k,
                                                                      const int32_t *__restrict__ counts,
                                                                      int32_t *offsets, int4 *items, uint32_t *n_items,
-                                                                     int4 *tc_items, uint32_t *n_tc_items) {
+                                                                     int4 *tc_items, uint32_t *n_tc_items, int tc_n) {
   __shared__ int warp_sums[33];
   // thread i owns experts [i * per, (i + 1) * per)
   const int per = (E + kScanThreads - 1) / kScanThreads;
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int 
     const int c = counts[i];
     my_cnt += c;
     my_items += (c + 7) >> 3;
-    my_tc += (c + 63) >> 6;
+    my_tc += (c + tc_n - 1) / tc_n;
   }
   int tot_cnt, tot_items, tot_tc;
   int pos = block_exclusive_scan(my_cnt, warp_sums, tot_cnt);
@@ -388,15 +388,15 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int 
     const int c = counts[i];
     offsets[i] = pos;
     for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
-    for (int j = 0; j < c; j += 64) tc_items[itc++] = make_int4(i, pos + j, min(64, c - j), 0);
+    for (int j = 0; j < c; j += tc_n) tc_items[itc++] = make_int4(i, pos + j, min(tc_n, c - j), 0);
     pos += c;
   }
   // the shared expert's items follow the routed ones
-  const int shared_items = (T + 7) >> 3, shared_tc = (T + 63) >> 6;
+  const int shared_items = (T + 7) >> 3, shared_tc = (T + tc_n - 1) / tc_n;
   for (int i = threadIdx.x; i < shared_items; i += blockDim.x)
     items[tot_items + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
   for (int i = threadIdx.x; i < shared_tc; i += blockDim.x)
-    tc_items[tot_tc + i] = make_int4(E, T * k + 64 * i, min(64, T - 64 * i), 0);
+    tc_items[tot_tc + i] = make_int4(E, T * k + tc_n * i, min(tc_n, T - tc_n * i), 0);
   if (threadIdx.x == 0) {
     offsets[E] = tot_cnt;  // == T * k when every index was valid
     *n_items = (uint32_t)(tot_items + shared_items);
@@ -462,7 +462,7 @@ cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaS
   const int wthreads = std::min(kScanThreads, (ws.words + 31) & ~31);
   dispatch_wscan_kernel<<<E, wthreads, 0, s>>>(ws.bitmap, ws.words, ws.wprefix, ws.counts);
   dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(E, T, k, ws.counts, ws.offsets, ws.items, ws.n_items, ws.tc_items,
-                                                  ws.n_tc_items);
+                                                  ws.n_tc_items, ws.tc_item_tokens > 0 ? ws.tc_item_tokens : 64);
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, true, s);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;

@@ -248,116 +248,4 @@ __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, i
   w_out = topk_softmax(key_float((uint32_t)(mine >> 32)), lane, k);
 }
 
-// Top-k keys of one slice of a token's logits, for a top-k split over several
-// warps: row[0 .. n) holds the logits of experts base .. base + n - 1.
-// Returns the key (float_key(logit) << 32 | ~expert) of rank `lane` within
-// the slice, 0 for lane >= k or past the slice's last value.  Threshold,
-// filter and rank as in warp_topk_fast (the threshold never admits the empty
-// key 0); when more than 32 values pass, k rounds of a warp arg-max on the
-// keys.  `scratch` is 64 uint64 of shared memory private to the warp.
-template <int NPL, bool kSmem>
-__device__ __forceinline__ uint64_t warp_topk_key(const float *row, int n, int base, int k, int lane,
-                                                  uint64_t *scratch) {
-  uint32_t kv[NPL];
-  uint32_t mk = 0;
-#pragma unroll
-  for (int j = 0; j < NPL; ++j) {
-    const int e = lane + 32 * j;
-    kv[j] = e < n ? float_key(load_logit<kSmem>(row, e)) : 0u;
-    mk = kv[j] > mk ? kv[j] : mk;
-  }
-  uint32_t *lmax = reinterpret_cast<uint32_t *>(scratch + 32);
-  lmax[lane] = mk;
-  __syncwarp();
-  int ge = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 q = reinterpret_cast<const uint4 *>(lmax)[i];
-    ge += (q.x >= mk) + (q.y >= mk) + (q.z >= mk) + (q.w >= mk);
-  }
-  uint32_t L = __reduce_max_sync(0xffffffffu, ge >= k ? mk : 0u);
-  L = L ? L : 1u;  // never the empty key
-  int cnt = 0;
-#pragma unroll
-  for (int j = 0; j < NPL; ++j) cnt += kv[j] >= L;
-  const int total = __reduce_add_sync(0xffffffffu, cnt);
-  __syncwarp();
-  if (total > 32) {
-    uint64_t key[NPL];
-#pragma unroll
-    for (int j = 0; j < NPL; ++j) key[j] = kv[j] ? ((uint64_t)kv[j] << 32) | (uint32_t)~(base + lane + 32 * j) : 0ull;
-    uint64_t mine = 0ull;
-    for (int r = 0; r < k; ++r) {
-      uint64_t best = 0ull;
-#pragma unroll
-      for (int j = 0; j < NPL; ++j) best = key[j] > best ? key[j] : best;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
-        best = o > best ? o : best;
-      }
-      if (lane == r) mine = best;
-#pragma unroll
-      for (int j = 0; j < NPL; ++j)
-        if (key[j] == best) key[j] = 0ull;
-    }
-    return mine;
-  }
-  int pos = cnt;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, pos, off);
-    if (lane >= off) pos += v;
-  }
-  pos -= cnt;
-#pragma unroll
-  for (int j = 0; j < NPL; ++j)
-    if (kv[j] >= L) scratch[pos++] = ((uint64_t)kv[j] << 32) | (uint32_t)~(base + lane + 32 * j);
-  __syncwarp();
-  const uint64_t cand = lane < total ? scratch[lane] : 0ull;
-  int r = 0;
-#pragma unroll
-  for (int o = 0; o < 32; o += 2) {
-    const ulonglong2 q = reinterpret_cast<const ulonglong2 *>(scratch)[o >> 1];
-    r += (o < total && q.x > cand) + (o + 1 < total && q.y > cand);
-  }
-  __syncwarp();
-  if (lane < k) scratch[32 + lane] = 0ull;
-  __syncwarp();
-  if (lane < total && r < k) scratch[32 + r] = cand;
-  __syncwarp();
-  const uint64_t mine = lane < k ? scratch[32 + lane] : 0ull;
-  __syncwarp();
-  return mine;
-}
-
-// Merge of the slices' candidates: `cand` holds n <= 128 keys (0 = empty);
-// returns the key of overall rank `lane` (lane < k).  Keys are distinct
-// (the expert index is part of the key), so ranking by counting is exact.
-__device__ __forceinline__ uint64_t warp_merge_keys(const uint64_t *cand, int n, int k, int lane,
-                                                    uint64_t *scratch) {
-  uint64_t c[4];
-  int r[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    c[j] = lane + 32 * j < n ? cand[lane + 32 * j] : 0ull;
-    r[j] = 0;
-  }
-  for (int i = 0; i < n; i += 2) {
-    const ulonglong2 q = *reinterpret_cast<const ulonglong2 *>(cand + i);
-    const bool has1 = i + 1 < n;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) r[j] += (q.x > c[j]) + (has1 && q.y > c[j]);
-  }
-  if (lane < k) scratch[lane] = 0ull;
-  __syncwarp();
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    if (c[j] && r[j] < k) scratch[r[j]] = c[j];
-  __syncwarp();
-  const uint64_t mine = lane < k ? scratch[lane] : 0ull;
-  __syncwarp();
-  return mine;
-}
-
 }  // namespace moe

@@ -95,6 +95,18 @@ def test_config2_prefill_chunk(full):
     print(f"config2: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
 
 
+@pytest.mark.parametrize("T", [600, 1500])
+def test_prefill_many_tokens_per_expert(T):
+    """Experts averaging 64 or more tokens take the one-tile, 128-token work items (ragged last items)."""
+    cfg = MoeConfig("many", 256, 128, 16, 2, T, "zipf")
+    L, w = build_layer(cfg, seed=7)
+    x = make_x(T, 256, seed=T)
+    y, idx, wts = gpu_forward(L, x)
+    err, l2, flagged = check_layer(cfg, w, x, y, idx, wts)
+    print(f"many-token items T={T}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+    assert l2 < 5e-3
+
+
 def test_prefill_ragged_and_cold_tail():
     cfg = MoeConfig("cold", 2048, 512, 512, 10, 133, "zipf_cold")
     L, w = build_layer(cfg, seed=1)
