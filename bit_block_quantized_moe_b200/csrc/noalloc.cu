@@ -1,9 +1,11 @@
 // moe_route_noalloc: routing for callers that cannot allocate device memory.
 //
-// Same router and top-k kernels as moe_route, but the scratch they need (the
-// [T, n_experts] fp32 router logits) is a file-scope device array of this
-// library instead of a caller-provided workspace.  Every GPU that loads the
-// library holds the array until the process exits.
+// The router and top-k kernels of moe_route (for more than 8 tokens the
+// legacy-MMA router, since the tcgen05 one keeps its split weights in the
+// workspace), but the scratch they need (the [T, n_experts] fp32 router
+// logits) is a file-scope device array of this library instead of a
+// caller-provided workspace.  Every GPU that loads the library holds the
+// array until the process exits.
 #include <mutex>
 
 #include "kernels.cuh"

@@ -131,11 +131,16 @@ moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_router *
  * device memory is reserved up front by their own pool, with nothing left to
  * hand out; and latency-bound loops that cannot afford an allocation's
  * implicit device synchronisation.
- * It computes exactly what moe_route computes (same kernels, same results),
- * but the scratch those kernels need -- the [T, n_experts] fp32 router logits
- * -- lives in a file-scope device array of MOE_NOALLOC_MAX_LOGITS floats
- * (1 MiB) inside this library, which every GPU that loads the library holds
- * until the process exits.  The call allocates nothing.
+ * It computes what moe_route computes.  For T <= 8 it runs the same kernels
+ * and returns identical results.  For more tokens moe_route's tcgen05 router
+ * needs the split router weights in its workspace, so this entry point uses
+ * the legacy-MMA router on the same exact weight split instead.  Its fp32
+ * sums run in a different order, so near-tied logits may select or order
+ * differently.  The scratch these kernels need -- the [T, n_experts] fp32
+ * router logits -- lives in a file-scope device array of
+ * MOE_NOALLOC_MAX_LOGITS floats (1 MiB) inside this library, which every GPU
+ * that loads the library holds until the process exits.  The call allocates
+ * nothing.
  *  - T * n_experts > MOE_NOALLOC_MAX_LOGITS returns MOE_ERR_WORKSPACE.
  *  - The first call on each device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
