@@ -32,6 +32,9 @@
 // d * (q - 1) and the 128 bias start the accumulator at minus the weighted
 // block sum of the token; the fp16 block scale d multiplies each block's fp32
 // result.  All products are exact.  Every wait is bounded (sync.cuh).
+#include <atomic>
+#include <mutex>
+
 #include "kernels.cuh"
 #include "router.cuh"
 #include "sync.cuh"
@@ -552,6 +555,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
 }
 
+// Per-device launch facts of the fused decode kernel.
+constexpr int kMaxDevices = 64;
+struct LaunchCache {
+  std::atomic<int> n_sm{0}, max_smem{0};
+  std::atomic<uint32_t> checked_smem{0};  // shared-memory size whose residency was checked (0: none)
+  uint32_t smem_attr = 0;                 // largest dynamic shared memory opted into (under mu)
+  std::mutex mu;
+};
+LaunchCache g_launch_cache[kMaxDevices];
+
 }  // namespace
 
 bool decode_fused_supported(const moe_dims &d, int T) {
@@ -574,11 +587,19 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
                                 const uint8_t *experts, const uint8_t *shared, int T, const Workspace &ws,
                                 int32_t *idx_out, float *w_out, uint16_t *out, cudaStream_t s) {
   const PackedGeom G = packed_geom(d.hidden, d.inter);
-  int dev = 0, n_sm = 0, max_smem = 0;
+  int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  LaunchCache &lc = g_launch_cache[dev];
+  int n_sm = lc.n_sm.load(std::memory_order_acquire), max_smem = lc.max_smem.load(std::memory_order_acquire);
+  if (n_sm == 0) {  // device properties, queried once per device
+    if ((err = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess ||
+        (err = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return err;
+    lc.max_smem.store(max_smem, std::memory_order_release);
+    lc.n_sm.store(n_sm, std::memory_order_release);
+  }
   const uint32_t stage_bytes = (uint32_t)max(G.gu_unit_bytes, 4 * G.dn_unit_bytes);
   const SmemLayout L0 = smem_layout(T, G.H, 0, stage_bytes);
   const int slots = (int)((max_smem - (int)L0.ring - 128) / (int)stage_bytes);
@@ -618,12 +639,21 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   a.stage_bytes = stage_bytes;
 
   void (*kern)(DecodeArgs) = decode_fused_kernel;
-  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
-  if (err != cudaSuccess) return err;
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, L.total);
-  if (err != cudaSuccess) return err;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  // The shared-memory opt-in and the residency check are done once per device and shared-memory size
+  // (they depend on nothing else), not on every call.
+  if (lc.checked_smem.load(std::memory_order_acquire) != L.total) {
+    std::lock_guard<std::mutex> lock(lc.mu);
+    if (L.total > lc.smem_attr) {
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+      if (err != cudaSuccess) return err;
+      lc.smem_attr = L.total;
+    }
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, L.total);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    lc.checked_smem.store(L.total, std::memory_order_release);
+  }
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(n_sm);

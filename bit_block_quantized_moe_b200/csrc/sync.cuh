@@ -37,8 +37,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Waits in hardware (the thread is suspended, it does not spin) until the
-// phase with the given parity completes or about 0.5 ms pass.
+// One hardware wait for the phase with the given parity: the thread may be
+// suspended until the phase completes or a system-dependent time limit passes;
+// true once the phase has completed.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
