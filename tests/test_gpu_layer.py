@@ -49,7 +49,7 @@ def test_config0_exact_workload(tiny):
 
 
 @pytest.mark.parametrize("dims", [(384, 256, 8, 3), (256, 128, 1, 1), (256, 128, 16, 16), (128, 384, 32, 5),
-                                  (1024, 128, 64, 8)])
+                                  (1024, 128, 64, 8), (512, 512, 16, 2)])
 def test_odd_shapes(dims):
     H, I, E, k = dims
     cfg = MoeConfig("t", H, I, E, k, 13, "zipf")
