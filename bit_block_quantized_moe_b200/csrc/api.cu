@@ -60,9 +60,9 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_tcnt = take(fused ? decode_counter_words(d) * 4 : 0);
   const size_t o_part = take(fused ? decode_partial_floats(d, T) * 4 : 0);
   const bool rtc = router_tc_supported(d, T);
-  const int rks = rtc ? router_tc_ksplit(d, T) : 1;
   const size_t o_wsplit = take(rtc ? (size_t)3 * E * H * 2 : 0);
-  const size_t o_rpart = take(rks > 1 ? (size_t)rks * T * E * 4 : 0);
+  // sized by the bound on every T (the split count falls as T grows), so that a workspace sized for max_T fits
+  const size_t o_rpart = take(rtc ? router_tc_partial_bytes_max() : 0);
   if (base && ws) {
     uint8_t *b = static_cast<uint8_t *>(base);
     ws->status = reinterpret_cast<uint32_t *>(b + o_hdr);

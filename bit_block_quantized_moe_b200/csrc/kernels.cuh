@@ -64,6 +64,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
                                 int32_t *idx_out, float *w_out, uint16_t *out, cudaStream_t s);
 bool router_tc_supported(const moe_dims &d, int T);
 int router_tc_ksplit(const moe_dims &d, int T);
+size_t router_tc_partial_bytes_max();
 cudaError_t launch_router_tc(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias, int T,
                              const Workspace &ws, cudaStream_t s);
 cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,

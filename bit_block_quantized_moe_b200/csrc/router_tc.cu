@@ -245,6 +245,10 @@ int router_tc_ksplit(const moe_dims &d, int T) {
   return ks;
 }
 
+// K-split partials never exceed one wave of tiles: ksplit x tiles <= kRtWave, so ksplit x T x E <= kRtWave x
+// kRtM x kRtN.  Sizing the workspace with this bound keeps moe_workspace_bytes(max_T) valid for every T <= max_T.
+size_t router_tc_partial_bytes_max() { return (size_t)kRtWave * kRtM * kRtN * 4; }
+
 size_t router_tc_smem_bytes() { return (size_t)kRtStages * kRtStageBytes + sizeof(RtBars) + 1024; }
 
 cudaError_t launch_router_tc(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias, int T,

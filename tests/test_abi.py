@@ -79,3 +79,16 @@ def test_host_checks_before_launch(lib):
     assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 2, 0x2004, 1 << 20, None) == 2
     assert lib.moe_rmsnorm_residual(None, None, None, 0, 256, 1e-6, None) == 0
     assert lib.moe_rmsnorm_residual(None, None, None, 4, 256, 1e-6, None) == 1
+
+
+@pytest.mark.parametrize("dims", [(2048, 512, 512, 10), (256, 128, 16, 2), (512, 512, 16, 2), (4096, 4096, 4096, 32),
+                                  (256, 1024, 4096, 8)])
+def test_workspace_size_never_shrinks_with_tokens(lib, dims):
+    """A workspace sized for max_T must hold every call with T <= max_T (the router's K-split count and the
+    prefill item size change with T, so this is not automatic)."""
+    d = B.moe_dims(*dims)
+    prev = 0
+    for T in list(range(1, 300)) + [511, 512, 513, 1023, 1024, 1025, 2048, 3277, 4096, 8192, 32768]:
+        need = lib.moe_workspace_bytes(ctypes.byref(d), T)
+        assert need >= prev, (dims, T, need, prev)
+        prev = need
