@@ -230,10 +230,13 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
   if (topk_idx_out) ws.idx = topk_idx_out;
   if (topk_w_out) ws.w = topk_w_out;
   if (decode_fused_supported(*dims, T)) {
+    // The fused kernel writes the routing copies as a pair (both pointers or neither): when only one is
+    // requested, the other goes to the workspace's own [T, top_k] buffer.
+    const bool copies = topk_idx_out || topk_w_out;
     return cuda_status(launch_decode_fused(*dims, x, router->w, router->bias,
                                            static_cast<const uint8_t *>(experts->packed),
-                                           static_cast<const uint8_t *>(shared->packed), T, ws, topk_idx_out,
-                                           topk_w_out, out, s));
+                                           static_cast<const uint8_t *>(shared->packed), T, ws,
+                                           copies ? ws.idx : nullptr, copies ? ws.w : nullptr, out, s));
   }
   cudaError_t err = launch_route(*dims, x, router->w, router->bias, T, ws, true, s);
   if (err == cudaSuccess) err = run_experts(*dims, x, experts, shared, out, T, ws, s, true);

@@ -215,6 +215,23 @@ def test_fused_decode_agrees_with_route_and_general_path(full):
     assert np.max(np.abs(yg - y1)) <= 4e-3 * np.max(np.abs(y1))
 
 
+def test_routing_copies_one_at_a_time(full):
+    """moe_layer_forward asked for only one of the two routing copies (the fused decode path writes them as a
+    pair; the other goes to the workspace)."""
+    L, w = full
+    x = make_x(3, 2048, seed=91)
+    xd = to_dev_bf16(x)
+    ridx, rw = L.route(xd)
+    idx = torch.full((3, 10), -1, dtype=torch.int32, device="cuda")
+    y1 = L.forward(xd, topk_idx=idx)
+    wts = torch.zeros((3, 10), dtype=torch.float32, device="cuda")
+    y2 = L.forward(xd, topk_w=wts)
+    torch.cuda.synchronize()
+    L.check_status()
+    assert torch.equal(idx, ridx) and torch.equal(wts, rw)
+    assert torch.equal(y1, y2)
+
+
 def test_config3_stack_layer_by_layer():
     """48-layer stack (config 3), checked on its first 3 seeded layers: x_0 = x; layer l
     reads bf16(RMSNorm(resid_l)); resid_{l+1} = resid_l + y_l (fp32 on the GPU).  Each
