@@ -56,13 +56,13 @@ class MoeConfig:
 
 
 CONFIGS = {
-    0: MoeConfig("tiny layer H256 I128 E16 top2+1 T8", 256, 128, 16, 2, 8),
-    1: MoeConfig("decode layer H2048 I512 E512 top10+1 T3", 2048, 512, 512, 10, 3),
-    2: MoeConfig("prefill layer H2048 I512 E512 top10+1 T1024 zipf", 2048, 512, 512, 10, 1024, "zipf"),
-    3: MoeConfig("48-layer stack H2048 I512 E512 top10+1 T1024 zipf rmsnorm", 2048, 512, 512, 10, 1024,
-                 "zipf", layers=48, rmsnorm=True),
-    4: MoeConfig("4-layer prefill H2048 I512 E512 top10+1 T32768 zipf", 2048, 512, 512, 10, 32768,
-                 "zipf", layers=4),
+    "tiny": MoeConfig("tiny layer H256 I128 E16 top2+1 T8", 256, 128, 16, 2, 8),
+    "decode": MoeConfig("decode layer H2048 I512 E512 top10+1 T3", 2048, 512, 512, 10, 3),
+    "prefill": MoeConfig("prefill layer H2048 I512 E512 top10+1 T1024 zipf", 2048, 512, 512, 10, 1024, "zipf"),
+    "stack": MoeConfig("48-layer stack H2048 I512 E512 top10+1 T1024 zipf rmsnorm", 2048, 512, 512, 10, 1024,
+                       "zipf", layers=48, rmsnorm=True),
+    "prefill_32k": MoeConfig("4-layer prefill H2048 I512 E512 top10+1 T32768 zipf", 2048, 512, 512, 10, 32768,
+                             "zipf", layers=4),
 }
 
 

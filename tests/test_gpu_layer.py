@@ -24,12 +24,12 @@ def _built():
 
 @pytest.fixture(scope="module")
 def tiny():
-    return build_layer(CONFIGS[0])
+    return build_layer(CONFIGS["tiny"])
 
 
 @pytest.fixture(scope="module")
 def full():
-    return build_layer(CONFIGS[2])  # full-size layer with the Zipf router bias
+    return build_layer(CONFIGS["prefill"])  # full-size layer with the Zipf router bias
 
 
 @pytest.mark.parametrize("T", [1, 2, 3, 7, 8, 9, 33, 100, 257])
@@ -37,15 +37,15 @@ def test_tiny_layer_all_tokens(tiny, T):
     L, w = tiny
     x = make_x(T, 256, seed=100 + T)
     y, idx, wts = gpu_forward(L, x)
-    err, l2, flagged = check_layer(CONFIGS[0], w, x, y, idx, wts)
+    err, l2, flagged = check_layer(CONFIGS["tiny"], w, x, y, idx, wts)
     assert l2 < 5e-3
 
 
-def test_config0_exact_workload(tiny):
+def test_tiny_layer_exact_workload(tiny):
     L, w = tiny
-    x = make_x(CONFIGS[0], seed=0)
+    x = make_x(CONFIGS["tiny"], seed=0)
     y, idx, wts = gpu_forward(L, x)
-    check_layer(CONFIGS[0], w, x, y, idx, wts)
+    check_layer(CONFIGS["tiny"], w, x, y, idx, wts)
 
 
 @pytest.mark.parametrize("dims", [(384, 256, 8, 3), (256, 128, 1, 1), (256, 128, 16, 16), (128, 384, 32, 5),
@@ -62,7 +62,7 @@ def test_odd_shapes(dims):
 
 def test_decode_window_full_size(full):
     L, w = full
-    cfg = CONFIGS[1]
+    cfg = CONFIGS["decode"]
     for T in (1, 2, 3):
         x = make_x(T, cfg.hidden, seed=7)
         y, idx, wts = gpu_forward(L, x)
@@ -70,17 +70,17 @@ def test_decode_window_full_size(full):
         print(f"T={T}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
 
 
-def test_config1_uniform_router():
-    cfg = CONFIGS[1]
+def test_decode_layer_uniform_router():
+    cfg = CONFIGS["decode"]
     L, w = build_layer(cfg)
     x = make_x(cfg, seed=0)
     y, idx, wts = gpu_forward(L, x)
     err, l2, flagged = check_layer(cfg, w, x, y, idx, wts)
-    print(f"config1: max-rel {err:.3e} relL2 {l2:.3e}")
+    print(f"decode layer: max-rel {err:.3e} relL2 {l2:.3e}")
 
 
-def test_config2_prefill_chunk(full):
-    cfg = CONFIGS[2]
+def test_prefill_chunk_1024(full):
+    cfg = CONFIGS["prefill"]
     L, w = full
     x = make_x(cfg, seed=0)
     y, idx, wts = gpu_forward(L, x)
@@ -92,7 +92,7 @@ def test_config2_prefill_chunk(full):
     sample = np.union1d(rng.choice(cfg.tokens, 192, replace=False), np.array(flagged, dtype=np.int64))
     sample = np.union1d(sample, [0, cfg.tokens - 1])
     err, l2, _ = check_layer(cfg, w, x, y, idx, wts, tokens=sample)
-    print(f"config2: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+    print(f"prefill chunk 1024: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
 
 
 @pytest.mark.parametrize("T", [600, 1500])
@@ -117,7 +117,7 @@ def test_prefill_ragged_and_cold_tail():
 
 def test_route_entry_point(full):
     L, w = full
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["prefill"]
     for T in (3, 1024):
         x = make_x(T, cfg.hidden, seed=11)
         idx, wts = L.route(to_dev_bf16(x))
@@ -159,7 +159,7 @@ def test_rmsnorm_residual():
 
 def test_experts_forward_given_routing(tiny):
     L, w = tiny
-    cfg = CONFIGS[0]
+    cfg = CONFIGS["tiny"]
     T = 21
     x = make_x(T, 256, seed=3)
     rng = np.random.default_rng(0)
@@ -194,7 +194,7 @@ def test_fused_decode_window_sizes(full, T):
     L, w = full
     x = make_x(T, 2048, seed=40 + T)
     y, idx, wts = gpu_forward(L, x)
-    err, l2, flagged = check_layer(CONFIGS[2], w, x, y, idx, wts)
+    err, l2, flagged = check_layer(CONFIGS["prefill"], w, x, y, idx, wts)
     print(f"fused T={T}: max-rel {err:.3e} relL2 {l2:.3e}")
 
 
@@ -232,8 +232,8 @@ def test_routing_copies_one_at_a_time(full):
     assert torch.equal(y1, y2)
 
 
-def test_config3_stack_layer_by_layer():
-    """48-layer stack (config 3), checked on its first 3 seeded layers: x_0 = x; layer l
+def test_stack_48_layers_first_three():
+    """48-layer stack, checked on its first 3 seeded layers: x_0 = x; layer l
     reads bf16(RMSNorm(resid_l)); resid_{l+1} = resid_l + y_l (fp32 on the GPU).  Each
     step is compared on 256 sampled tokens: the GPU's RMSNorm output against the
     oracle's RMSNorm of the GPU residual, and the GPU layer against the oracle layer on
@@ -242,7 +242,7 @@ def test_config3_stack_layer_by_layer():
     bench's workload."""
     from bit_block_quantized_moe_b200 import moe_rmsnorm_residual
 
-    cfg = CONFIGS[3]
+    cfg = CONFIGS["stack"]
     T, H = cfg.tokens, cfg.hidden
     rng = np.random.default_rng(3)
     sample = np.sort(rng.choice(T, 256, replace=False))
@@ -270,12 +270,12 @@ def test_config3_stack_layer_by_layer():
         del L
 
 
-def test_config4_prefill_32k(full):
-    """Config 4: a T = 32768 prefill chunk through a full-size Zipf layer: routing of
+def test_prefill_chunk_32768(full):
+    """A T = 32768 prefill chunk through a full-size Zipf layer: routing of
     every token against the oracle, outputs on 256 sampled tokens (plus the flagged
     ones and both ends).  The decode sweep T in {1, 2, 3} on the same weights is
     test_decode_window_full_size."""
-    cfg = CONFIGS[4]
+    cfg = CONFIGS["prefill_32k"]
     L, w = full
     x = make_x(cfg, seed=4)
     y, idx, wts = gpu_forward(L, x)
@@ -285,4 +285,4 @@ def test_config4_prefill_32k(full):
     sample = np.union1d(rng.choice(cfg.tokens, 256, replace=False), np.array(flagged, dtype=np.int64))
     sample = np.union1d(sample, [0, cfg.tokens - 1])
     err, l2, _ = check_layer(cfg, w, x, y, idx, wts, tokens=sample)
-    print(f"config4 T=32768: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+    print(f"prefill chunk 32768: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")

@@ -6,7 +6,7 @@ from gen import CONFIGS, make_expert, make_router, make_x, canonical_expert_byte
 
 
 def test_shapes_and_determinism():
-    cfg = CONFIGS[0]
+    cfg = CONFIGS["tiny"]
     x1, x2 = make_x(cfg, seed=0), make_x(cfg, seed=0)
     assert x1.shape == (8, 256) and x1.dtype == np.uint16 and np.array_equal(x1, x2)
     assert not np.array_equal(x1, make_x(cfg, seed=1))
@@ -28,7 +28,7 @@ def test_code_and_scale_distribution():
 
 def test_zipf_skew_at_prefill_chunk():
     # T=1024, top-10 of 512: the hottest expert near 100 slots, every expert hit.
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["prefill"]
     Wr, b = make_router(cfg, seed=0)
     idx, w, gap, _ = oracle.route(make_x(cfg, seed=0), Wr, b, cfg.top_k)
     c = np.bincount(idx.ravel(), minlength=cfg.n_experts)
@@ -36,5 +36,5 @@ def test_zipf_skew_at_prefill_chunk():
     assert 80 <= c.max() <= 130
     assert c.min() >= 1
     # uniform routing at decode: bias zero
-    Wr1, b1 = make_router(CONFIGS[1], seed=0)
+    Wr1, b1 = make_router(CONFIGS["decode"], seed=0)
     assert np.all(b1 == 0)

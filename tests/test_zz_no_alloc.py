@@ -25,7 +25,7 @@ def test_noalloc_route_matches_workspace_route():
     import bit_block_quantized_moe_b200 as M
     from bit_block_quantized_moe_b200 import binding as B
 
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["prefill"]
     dims = M.moe_dims(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k)
     Wr, b = make_router(cfg, seed=0)
     Wd, bd = torch.from_numpy(Wr).cuda(), torch.from_numpy(b).cuda()
