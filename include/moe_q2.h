@@ -111,7 +111,10 @@ moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_ex
  * kernel's grid-barrier counter (offset 64): zero the workspace (or at least
  * those 256 bytes) once after allocating it, and again after a call reported
  * MOE_ERR_TIMEOUT.  One workspace must not be used by two calls that can run
- * at the same time. */
+ * at the same time.  A workspace of moe_workspace_bytes(dims, max_T) serves
+ * every T <= max_T.  For T > 8 it also holds the router weights split into
+ * three bf16 planes (3 * n_experts * hidden * 2 bytes) and the router's K-split
+ * partial sums (at most 4.85 MB). */
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T);
 
 /* ---- routing ------------------------------------------------------------------
