@@ -6,6 +6,9 @@
 // logits) is a file-scope device array of this library instead of a
 // caller-provided workspace.  Every GPU that loads the library holds the
 // array until the process exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "kernels.cuh"
@@ -17,24 +20,73 @@ constexpr size_t kNoAllocLogits = MOE_NOALLOC_MAX_LOGITS;  // 1 MiB of fp32 logi
 static __device__ __align__(256) float g_noalloc_logits[kNoAllocLogits];
 
 constexpr int kMaxDevices = 64;
+
+// Device address of the array, looked up with the device current and kept per
+// device together with the id of the CUDA context it belongs to: a device
+// reset ends that context (and the module image holding the array), so a call
+// made in a new context looks the address up again.
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;
+  float *ptr = nullptr;
+};
 std::mutex g_lookup_mutex;
-float *g_scratch[kMaxDevices];  // device address of the array, looked up once per device
+ScratchAddr g_scratch[kMaxDevices];
+
+// Driver entry points for the current context's id (through the runtime, so
+// the library needs no link against the driver library).
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+  bool ok = false;
+};
+const CtxFns &ctx_fns() {
+  static CtxFns f = [] {
+    CtxFns r;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      r.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      r.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    r.ok = r.get_current && r.get_id;
+    return r;
+  }();
+  return f;
+}
+
+cudaError_t current_ctx_id(unsigned long long *id) {
+  const CtxFns &f = ctx_fns();
+  if (!f.ok) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorInvalidContext;
+  return f.get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidContext;
+}
 
 // The array's name is only a host-side stand-in in host code; the kernels get
-// its device address, looked up once per device with that device current.
+// its device address, looked up once per device and context with that device
+// current.
 cudaError_t scratch_for_current_device(float **out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_lookup_mutex);
-  if (!g_scratch[dev]) {
+  unsigned long long id = 0;
+  // With no context current yet, the lookup below creates the device's primary context.
+  const bool have_ctx = current_ctx_id(&id) == cudaSuccess;
+  ScratchAddr &s = g_scratch[dev];
+  if (!have_ctx || !s.ptr || s.ctx_id != id) {
     void *p = nullptr;
     err = cudaGetSymbolAddress(&p, g_noalloc_logits);
     if (err != cudaSuccess) return err;
-    g_scratch[dev] = static_cast<float *>(p);
+    err = current_ctx_id(&id);
+    if (err != cudaSuccess) return err;
+    s.ptr = static_cast<float *>(p);
+    s.ctx_id = id;
   }
-  *out = g_scratch[dev];
+  *out = s.ptr;
   return cudaSuccess;
 }
 

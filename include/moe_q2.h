@@ -129,10 +129,10 @@ moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_router *
 
 /* ---- routing without a workspace --------------------------------------------------
  * The paper has no counterpart to this entry point; it exists for callers of
- * this library that cannot allocate device memory: code running inside a
- * stream capture, where a cudaMalloc would break the capture; engines whose
- * device memory is reserved up front by their own pool, with nothing left to
- * hand out; and latency-bound loops that cannot afford an allocation's
+ * this library that cannot allocate device memory: engines whose device
+ * memory is reserved up front by their own pool, with nothing left to hand
+ * out; plug-ins running inside a host framework that owns every device
+ * allocation; and latency-bound loops that cannot afford an allocation's
  * implicit device synchronisation.
  * It computes what moe_route computes.  For T <= 8 it runs the same kernels
  * and returns identical results.  For more tokens moe_route's tcgen05 router
@@ -147,6 +147,9 @@ moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_router *
  *  - T * n_experts > MOE_NOALLOC_MAX_LOGITS returns MOE_ERR_WORKSPACE.
  *  - The first call on each device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
+ *    The address is kept together with the id of the CUDA context it was
+ *    looked up in; after a device reset the first call in the new context
+ *    looks it up again (so that call, too, should come before any capture).
  *  - All calls share the one array: calls that overlap on the GPU (different
  *    streams, or different host threads) race and may return each other's
  *    routing.  Nothing in the array needs to start at zero: every call

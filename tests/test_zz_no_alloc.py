@@ -1,6 +1,7 @@
 """moe_route_noalloc: routing for callers that cannot allocate device memory
-(inside a stream capture, under a pre-reserved memory pool, or in loops that
-cannot afford an allocation's device synchronisation).  Its scratch is a static
+(engines whose device memory is reserved up front by their own pool, plug-ins
+inside a framework that owns every allocation, or loops that cannot afford an
+allocation's device synchronisation).  Its scratch is a static
 device array inside the library; this checks it and moe_route, which uses a
 caller-provided workspace, against the oracle on two calls in a row.  With more
 than 8 tokens the two entry points use different router kernels (the workspace
