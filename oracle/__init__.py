@@ -62,6 +62,9 @@ def lib():
         L.orc_layer.restype = i
         L.orc_layer.argtypes = [i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
         L.orc_rmsnorm.argtypes = [i, P, ctypes.c_double, P]
+        L.orc_stack.restype = i
+        L.orc_stack.argtypes = [i, i, i, i, i, i, P, P, P, P, P, ctypes.c_double, P, ctypes.c_double, P, P, P,
+                                ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         L.orc_num_threads.restype = i
         _lib = L
     return _lib
@@ -189,3 +192,38 @@ def rmsnorm(v: np.ndarray, eps: float = 1e-6) -> np.ndarray:
         lib().orc_rmsnorm(a.shape[1], _p(row), float(eps), _p(o))
         out[r] = o
     return out.reshape(np.shape(v))
+
+
+def stack(x_bits, layers, top_k: int, inter: int, eps: float = 1e-6, follow_idx=None, tie_gap: float = 1e-5):
+    """A stack of layers over bf16 tokens x [T, H]: r_0 = x; r_{l+1} = r_l + layer_l(bf16(RMSNorm(r_l))),
+    the residual in fp64.  ``layers`` is a list of dicts with router_w, router_b, experts, shared (as
+    gen.make_layer returns).  ``follow_idx`` [L, T, k] (optional): a routing made elsewhere that the stack
+    takes at near-ties (see orc_stack).  Returns (resid [T,H] fp64, idx [L,T,k], gap [L,T], n_followed,
+    n_mismatch)."""
+    x = _c(x_bits, np.uint16)
+    T, H = x.shape
+    L = len(layers)
+    keep = []
+
+    def arr(key, dtype):
+        vals = [None if lay[key] is None else _c(lay[key], dtype) for lay in layers]
+        keep.append(vals)
+        return (ctypes.c_void_p * max(L, 1))(*[None if v is None else v.ctypes.data for v in vals])
+
+    E = np.asarray(layers[0]["router_w"]).shape[0] if L else top_k  # no layers: nothing is routed
+    for lay in layers:
+        assert np.asarray(lay["experts"]).size == E * expert_bytes(H, inter)
+    rw, ex, sh = arr("router_w", np.float32), arr("experts", np.uint8), arr("shared", np.uint8)
+    rb = arr("router_b", np.float32) if L and all(lay["router_b"] is not None for lay in layers) else None
+    fi = _c(follow_idx, np.int32)
+    if fi is not None:
+        assert fi.shape == (L, T, top_k)
+    resid = np.empty((T, H), dtype=np.float64)
+    idx = np.empty((L, T, top_k), dtype=np.int32)
+    gap = np.empty((L, T), dtype=np.float64)
+    nf, nm = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib().orc_stack(H, inter, E, top_k, L, T, _p(x), rw, rb, ex, sh, float(eps), _p(fi), float(tie_gap),
+                         _p(resid), _p(idx), _p(gap), ctypes.byref(nf), ctypes.byref(nm))
+    if rc:
+        raise ValueError("oracle stack: bad dimensions")
+    return resid, idx, gap, nf.value, nm.value

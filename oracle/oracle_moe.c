@@ -18,7 +18,9 @@
  *   5. E_e(x) = Wd_e (silu(Wg_e x) * (Wu_e x)),  silu(z) = z / (1 + exp(-z))
  *   6. y = E_shared(x) + sum_{e in S} w[e] E_e(x)          (plus 1 shared expert,
  *      Strata tuning page, section 2 model table)
- * Everything is computed in binary64 with no intermediate rounding.  Steps the
+ *   7. (a stack of layers, orc_stack) r <- r + layer(bf16(RMSNorm(r))), r in binary64
+ * Everything is computed in binary64 with no intermediate rounding (the one
+ * exception: a stacked layer's input is rounded to bf16, the layer's input type).  Steps the
  * pages leave open (block bit layout, softmax placement, tie rule, shared-expert
  * weight, SwiGLU form) follow the readings listed in the design notes.
  */
@@ -261,6 +263,87 @@ void orc_rmsnorm(int n, const double *v, double eps, double *out) {
   for (int i = 0; i < n; ++i) ss += v[i] * v[i];
   double r = 1.0 / sqrt(ss / n + eps);
   for (int i = 0; i < n; ++i) out[i] = v[i] * r;
+}
+
+/* ---------- a stack of layers ------------------------------------------------
+ * The pages' model runs 48 such layers one after another (Strata tuning page,
+ * section 2 model table); between layers the stack keeps a residual stream and
+ * normalises the layer input (unit-gain RMSNorm, eps given):
+ *   r_0 = x
+ *   for l = 0 .. L-1:  u_l = bf16(RMSNorm(r_l));  r_{l+1} = r_l + layer_l(u_l)
+ * The residual r stays in binary64 here; the layer input u_l is rounded to
+ * bfloat16 (nearest even) because the layer consumes bf16 activations.  Each
+ * layer routes u_l exactly as orc_layer does.
+ * follow_idx (nullable, [L][tokens][top_k]): a routing made elsewhere.  Where
+ * its set for (layer, token) differs from this oracle's own and the oracle's
+ * k-th/(k+1)-th logit gap is below tie_gap, the stack takes that set (weights
+ * = softmax over its logits) so that both sides stay on one trajectory; such
+ * (layer, token) pairs are counted in *n_followed.  Where the sets differ with
+ * a larger gap the oracle keeps its own set and counts the pair in
+ * *n_mismatch.  idx_out [L][tokens][top_k] and gap_out [L][tokens] (nullable)
+ * receive the routing actually used and the oracle's own gap. */
+int orc_stack(int hidden, int inter, int n_experts, int top_k, int n_layers, int tokens, const uint16_t *x_bf16,
+              const float *const *router_w, const float *const *router_b, const uint8_t *const *experts,
+              const uint8_t *const *shared, double eps, const int32_t *follow_idx, double tie_gap, double *resid,
+              int32_t *idx_out, double *gap_out, int *n_followed, int *n_mismatch) {
+  if (top_k < 1 || top_k > n_experts || hidden % ORC_QBLOCK || inter % ORC_QBLOCK || n_layers < 0) return 1;
+  size_t ebytes = orc_expert_bytes(hidden, inter);
+  int followed = 0, mismatch = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : followed, mismatch)
+  for (int t = 0; t < tokens; ++t) {
+    double *r = resid + (size_t)t * hidden;
+    double *v = (double *)malloc(sizeof(double) * hidden);
+    double *u = (double *)malloc(sizeof(double) * hidden);
+    double *lg = (double *)malloc(sizeof(double) * n_experts);
+    double *y = (double *)malloc(sizeof(double) * hidden);
+    double *ye = (double *)malloc(sizeof(double) * hidden);
+    int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * top_k);
+    double *wt = (double *)malloc(sizeof(double) * top_k);
+    for (int h = 0; h < hidden; ++h) r[h] = orc_bf16_to_double(x_bf16[(size_t)t * hidden + h]);
+    for (int l = 0; l < n_layers; ++l) {
+      orc_rmsnorm(hidden, r, eps, v);
+      for (int h = 0; h < hidden; ++h) u[h] = orc_bf16_to_double(orc_double_to_bf16(v[h]));
+      double g = INFINITY;
+      orc_logits_one(hidden, n_experts, u, router_w[l], router_b ? router_b[l] : NULL, lg);
+      orc_topk_one(lg, n_experts, top_k, sel, wt, &g);
+      if (follow_idx) {
+        const int32_t *f = follow_idx + ((size_t)l * tokens + t) * top_k;
+        int same = 1;
+        for (int j = 0; j < top_k && same; ++j) {
+          int found = 0;
+          for (int i = 0; i < top_k; ++i) found |= f[i] == sel[j];
+          same = found;
+        }
+        if (!same) {
+          if (g < tie_gap) {
+            memcpy(sel, f, sizeof(int32_t) * top_k);
+            weights_for_set(lg, top_k, sel, wt);
+            ++followed;
+          } else {
+            ++mismatch;
+          }
+        }
+      }
+      orc_expert_forward(hidden, inter, shared[l], u, y); /* shared expert, weight 1 */
+      for (int j = 0; j < top_k; ++j) {
+        orc_expert_forward(hidden, inter, experts[l] + (size_t)sel[j] * ebytes, u, ye);
+        for (int h = 0; h < hidden; ++h) y[h] += wt[j] * ye[h];
+      }
+      for (int h = 0; h < hidden; ++h) r[h] += y[h];
+      if (idx_out) memcpy(idx_out + ((size_t)l * tokens + t) * top_k, sel, sizeof(int32_t) * top_k);
+      if (gap_out) gap_out[(size_t)l * tokens + t] = g;
+    }
+    free(v);
+    free(u);
+    free(lg);
+    free(y);
+    free(ye);
+    free(sel);
+    free(wt);
+  }
+  if (n_followed) *n_followed = followed;
+  if (n_mismatch) *n_mismatch = mismatch;
+  return 0;
 }
 
 int orc_num_threads(void) {
