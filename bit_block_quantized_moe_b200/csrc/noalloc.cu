@@ -60,8 +60,8 @@ cudaError_t current_ctx_id(unsigned long long *id) {
   const CtxFns &f = ctx_fns();
   if (!f.ok) return cudaErrorNotSupported;
   CUcontext ctx = nullptr;
-  if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorInvalidContext;
-  return f.get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidContext;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+  return f.get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
 }
 
 // The array's name is only a host-side stand-in in host code; the kernels get
