@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     moe_canonical_expert_bytes,
     moe_check_status,
     moe_dims,
+    moe_dispatch,
     moe_experts_forward,
     moe_layer_forward,
     moe_pack_q2,

@@ -45,6 +45,7 @@ EXPORTED = [
     "moe_route_noalloc",
     "moe_layer_forward",
     "moe_experts_forward",
+    "moe_dispatch",
     "moe_rmsnorm_residual",
     "moe_trace_kernel",
     "moe_check_status",
@@ -79,6 +80,8 @@ def lib():
         L.moe_experts_forward.restype = ctypes.c_int
         L.moe_experts_forward.argtypes = [D, P, P, P, ctypes.POINTER(moe_experts), ctypes.POINTER(moe_shared), P,
                                           i32, P, sz, P]
+        L.moe_dispatch.restype = ctypes.c_int
+        L.moe_dispatch.argtypes = [D, P, i32, P, P, P, P, P, sz, P]
         L.moe_rmsnorm_residual.restype = ctypes.c_int
         L.moe_rmsnorm_residual.argtypes = [P, P, P, i32, i32, ctypes.c_float, P]
         L.moe_trace_kernel.restype = ctypes.c_int
@@ -176,6 +179,13 @@ def moe_experts_forward(dims, x, topk_idx, topk_w, experts_packed, shared_packed
                                      ctypes.byref(ex), ctypes.byref(sh), _ptr(out), int(T), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "moe_experts_forward")
+
+
+def moe_dispatch(dims, topk_idx, T: int, counts, offsets, perm, inv, workspace, stream=None):
+    code = lib().moe_dispatch(ctypes.byref(_dims(dims)), _ptr(topk_idx), int(T), _ptr(counts), _ptr(offsets),
+                              _ptr(perm), _ptr(inv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(code, "moe_dispatch")
 
 
 def moe_rmsnorm_residual(resid, y, x_norm, T: int, hidden: int, eps: float = 1e-6, stream=None):

@@ -77,6 +77,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->idx = reinterpret_cast<int32_t *>(b + o_idx);
     ws->w = reinterpret_cast<float *>(b + o_w);
     ws->slot_pos = reinterpret_cast<int32_t *>(b + o_slot);
+    ws->perm = nullptr;
     ws->sorted_tok = reinterpret_cast<int32_t *>(b + o_stok);
     ws->sorted_w = reinterpret_cast<float *>(b + o_sw);
     ws->items = reinterpret_cast<int4 *>(b + o_items);
@@ -257,6 +258,29 @@ moe_status moe_experts_forward(const moe_dims *dims, const uint16_t *x, const in
   ws.idx = const_cast<int32_t *>(topk_idx);
   ws.w = const_cast<float *>(topk_w);
   return cuda_status(run_experts(*dims, x, experts, shared, out, T, ws, s, false));
+}
+
+moe_status moe_dispatch(const moe_dims *dims, const int32_t *topk_idx, int32_t T, int32_t *counts,
+                        int32_t *offsets, int32_t *perm, int32_t *inv, void *workspace, size_t ws_bytes,
+                        moe_stream_t stream) {
+  if (!dims_ok(dims) || T < 0) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !counts || !offsets || !perm || !inv || !workspace) return MOE_ERR_ARG;
+  if (!aligned16(workspace)) return MOE_ERR_ALIGN;
+  if (ws_bytes < workspace_layout(*dims, T, nullptr, nullptr)) return MOE_ERR_WORKSPACE;
+  const moe_status dev = device_ok();
+  if (dev != MOE_OK) return dev;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Workspace ws;
+  workspace_layout(*dims, T, workspace, &ws);
+  ws.idx = const_cast<int32_t *>(topk_idx);
+  ws.counts = counts;
+  ws.offsets = offsets;
+  ws.slot_pos = inv;
+  ws.perm = perm;
+  cudaError_t err = launch_dispatch_bits(*dims, T, ws, s);
+  if (err == cudaSuccess) err = launch_dispatch(*dims, T, ws, s);
+  return cuda_status(err);
 }
 
 moe_status moe_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int32_t T, int32_t hidden,

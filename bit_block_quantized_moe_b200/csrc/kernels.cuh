@@ -19,6 +19,7 @@ struct Workspace {
   int32_t *idx;            // [T][k]
   float *w;                // [T][k]
   int32_t *slot_pos;       // [T*k]: sorted position of slot (t, j)
+  int32_t *perm;           // optional [T*k]: slot t*k + j at each sorted position (moe_dispatch only)
   int32_t *sorted_tok;     // [T*k + T]: token of each sorted position (shared slots last)
   float *sorted_w;         // [T*k + T]
   int4 *items;             // [max_items]: (expert, first position, tokens <= 8, 0)

@@ -407,7 +407,8 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int 
 __global__ void dispatch_place_kernel(const int32_t *__restrict__ idx, const float *__restrict__ w, int T, int k,
                                       int E, int words, const uint32_t *__restrict__ bitmap,
                                       const uint32_t *__restrict__ wprefix, const int32_t *__restrict__ offsets,
-                                      int32_t *slot_pos, int32_t *sorted_tok, float *sorted_w, uint32_t *status) {
+                                      int32_t *slot_pos, int32_t *sorted_tok, float *sorted_w, int32_t *perm,
+                                      uint32_t *status) {
   const long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long routed = (long long)T * k;
   if (s >= routed + T) return;
@@ -424,6 +425,7 @@ __global__ void dispatch_place_kernel(const int32_t *__restrict__ idx, const flo
     slot_pos[s] = pos;
     sorted_tok[pos] = t;
     sorted_w[pos] = w[s];
+    if (perm) perm[pos] = (int32_t)s;
   } else {
     const int t = (int)(s - routed);
     sorted_tok[routed + t] = t;
@@ -470,7 +472,7 @@ cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaS
   trace_mark(MOE_KERNEL_DISPATCH_PLACE, false, s);
   dispatch_place_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ws.idx, ws.w, T, k, E, ws.words, ws.bitmap,
                                                                      ws.wprefix, ws.offsets, ws.slot_pos,
-                                                                     ws.sorted_tok, ws.sorted_w, ws.status);
+                                                                     ws.sorted_tok, ws.sorted_w, ws.perm, ws.status);
   trace_mark(MOE_KERNEL_DISPATCH_PLACE, true, s);
   return cudaGetLastError();
 }

@@ -184,6 +184,25 @@ moe_status moe_experts_forward(const moe_dims *dims, const uint16_t *x, const in
                                const float *topk_w, const moe_experts *experts, const moe_shared *shared,
                                uint16_t *out, int32_t T, void *workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* The dispatch step on its own, for a routing made elsewhere (the step the
+ * expert half of the layer starts with): the token-to-expert histogram, its
+ * exclusive scan and the stable permutation that groups the routed slots by
+ * expert.  Each token is routed to top_k experts (Strata tuning page, section
+ * 2 model table: 10 of 512 per token), so there are T * top_k slots; slot
+ * s = t * top_k + j holds topk_idx[t][j].  Outputs (device, int32):
+ *   counts [n_experts]      slots routed to each expert;
+ *   offsets [n_experts + 1] exclusive prefix sum of counts, offsets[n_experts] = T * top_k;
+ *   perm [T * top_k]        the slot at each sorted position: experts in ascending order, and within an
+ *                           expert the slots in ascending order (a stable sort of the slots by expert);
+ *   inv [T * top_k]         the sorted position of each slot (perm[inv[s]] == s).
+ * Indices must lie in [0, n_experts) and be distinct within a token; a slot
+ * with an index out of range sets MOE_ERR_DEVICE in the workspace status, is
+ * left out of the counts and gets inv = -1.  The workspace is the one
+ * moe_layer_forward takes (moe_workspace_bytes(dims, T) bytes). */
+moe_status moe_dispatch(const moe_dims *dims, const int32_t *topk_idx, int32_t T, int32_t *counts,
+                        int32_t *offsets, int32_t *perm, int32_t *inv, void *workspace, size_t ws_bytes,
+                        moe_stream_t stream);
+
 /* ---- between layers (a stack of layers) -------------------------------------------
  * resid [T, hidden] fp32 (in/out), y [T, hidden] bf16 (may be NULL),
  * x_norm [T, hidden] bf16 (out):

@@ -63,7 +63,7 @@ def lib():
         L.orc_layer.argtypes = [i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
         L.orc_rmsnorm.argtypes = [i, P, ctypes.c_double, P]
         L.orc_stack.restype = i
-        L.orc_stack.argtypes = [i, i, i, i, i, i, P, P, P, P, P, ctypes.c_double, P, ctypes.c_double, P, P, P,
+        L.orc_stack.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, ctypes.c_double, P, ctypes.c_double, P, P, P,
                                 ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         L.orc_num_threads.restype = i
         _lib = L
@@ -194,12 +194,13 @@ def rmsnorm(v: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     return out.reshape(np.shape(v))
 
 
-def stack(x_bits, layers, top_k: int, inter: int, eps: float = 1e-6, follow_idx=None, tie_gap: float = 1e-5):
+def stack(x_bits, layers, top_k: int, inter: int, eps: float = 1e-6, follow_idx=None, tie_gap: float = 1e-5,
+          resid_in=None):
     """A stack of layers over bf16 tokens x [T, H]: r_0 = x; r_{l+1} = r_l + layer_l(bf16(RMSNorm(r_l))),
     the residual in fp64.  ``layers`` is a list of dicts with router_w, router_b, experts, shared (as
     gen.make_layer returns).  ``follow_idx`` [L, T, k] (optional): a routing made elsewhere that the stack
     takes at near-ties (see orc_stack).  Returns (resid [T,H] fp64, idx [L,T,k], gap [L,T], n_followed,
-    n_mismatch)."""
+    n_mismatch).  ``resid_in`` [T, H] fp64 (optional): start from this residual instead of x."""
     x = _c(x_bits, np.uint16)
     T, H = x.shape
     L = len(layers)
@@ -218,11 +219,14 @@ def stack(x_bits, layers, top_k: int, inter: int, eps: float = 1e-6, follow_idx=
     fi = _c(follow_idx, np.int32)
     if fi is not None:
         assert fi.shape == (L, T, top_k)
+    r_in = _c(resid_in, np.float64)
+    if r_in is not None:
+        assert r_in.shape == (T, H)
     resid = np.empty((T, H), dtype=np.float64)
     idx = np.empty((L, T, top_k), dtype=np.int32)
     gap = np.empty((L, T), dtype=np.float64)
     nf, nm = ctypes.c_int(0), ctypes.c_int(0)
-    rc = lib().orc_stack(H, inter, E, top_k, L, T, _p(x), rw, rb, ex, sh, float(eps), _p(fi), float(tie_gap),
+    rc = lib().orc_stack(H, inter, E, top_k, L, T, _p(x), _p(r_in), rw, rb, ex, sh, float(eps), _p(fi), float(tie_gap),
                          _p(resid), _p(idx), _p(gap), ctypes.byref(nf), ctypes.byref(nm))
     if rc:
         raise ValueError("oracle stack: bad dimensions")

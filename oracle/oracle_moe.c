@@ -281,8 +281,12 @@ void orc_rmsnorm(int n, const double *v, double eps, double *out) {
  * (layer, token) pairs are counted in *n_followed.  Where the sets differ with
  * a larger gap the oracle keeps its own set and counts the pair in
  * *n_mismatch.  idx_out [L][tokens][top_k] and gap_out [L][tokens] (nullable)
- * receive the routing actually used and the oracle's own gap. */
+ * receive the routing actually used and the oracle's own gap.
+ * resid_in (nullable, [tokens][hidden]): start from this residual instead of
+ * x (so that a long stack can be run a few layers at a time; the layers of
+ * one token run in order either way, so the result is the same). */
 int orc_stack(int hidden, int inter, int n_experts, int top_k, int n_layers, int tokens, const uint16_t *x_bf16,
+              const double *resid_in,
               const float *const *router_w, const float *const *router_b, const uint8_t *const *experts,
               const uint8_t *const *shared, double eps, const int32_t *follow_idx, double tie_gap, double *resid,
               int32_t *idx_out, double *gap_out, int *n_followed, int *n_mismatch) {
@@ -299,7 +303,8 @@ int orc_stack(int hidden, int inter, int n_experts, int top_k, int n_layers, int
     double *ye = (double *)malloc(sizeof(double) * hidden);
     int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * top_k);
     double *wt = (double *)malloc(sizeof(double) * top_k);
-    for (int h = 0; h < hidden; ++h) r[h] = orc_bf16_to_double(x_bf16[(size_t)t * hidden + h]);
+    for (int h = 0; h < hidden; ++h)
+      r[h] = resid_in ? resid_in[(size_t)t * hidden + h] : orc_bf16_to_double(x_bf16[(size_t)t * hidden + h]);
     for (int l = 0; l < n_layers; ++l) {
       orc_rmsnorm(hidden, r, eps, v);
       for (int h = 0; h < hidden; ++h) u[h] = orc_bf16_to_double(orc_double_to_bf16(v[h]));

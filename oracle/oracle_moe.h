@@ -30,7 +30,7 @@ int orc_layer(int hidden, int inter, int n_experts, int top_k, int tokens, const
               const int32_t *forced_idx, double *y, int32_t *idx_out, double *w_out, double *gap_out);
 void orc_rmsnorm(int n, const double *v, double eps, double *out);
 int orc_stack(int hidden, int inter, int n_experts, int top_k, int n_layers, int tokens, const uint16_t *x_bf16,
-              const float *const *router_w, const float *const *router_b, const uint8_t *const *experts,
+              const double *resid_in, const float *const *router_w, const float *const *router_b, const uint8_t *const *experts,
               const uint8_t *const *shared, double eps, const int32_t *follow_idx, double tie_gap, double *resid,
               int32_t *idx_out, double *gap_out, int *n_followed, int *n_mismatch);
 int orc_num_threads(void);

@@ -77,6 +77,10 @@ def test_host_checks_before_launch(lib):
     assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 0, 0x2000, 0, None) == 0
     assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 2, 0x2000, 100, None) == 1    # output too small
     assert lib.moe_pack_q2(ctypes.byref(d), 0x1000, 2, 0x2004, 1 << 20, None) == 2
+    assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 0, None, None, None, None, None, 0, None) == 0  # T = 0
+    assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 4, 0x2000, 0x3000, None, 0x5000, 0x10000, ws, None) == 1
+    assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 4, 0x2000, 0x3000, 0x4000, 0x5000, 0x10004, ws, None) == 2
+    assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 9, 0x2000, 0x3000, 0x4000, 0x5000, 0x10000, 16, None) == 3
     assert lib.moe_rmsnorm_residual(None, None, None, 0, 256, 1e-6, None) == 0
     assert lib.moe_rmsnorm_residual(None, None, None, 4, 256, 1e-6, None) == 1
 

@@ -87,11 +87,8 @@ def test_prefill_chunk_1024(full):
     # routing: every token against the oracle
     idx_o, w_o, gap, _ = oracle.route(x, w["router_w"], w["router_b"], cfg.top_k)
     flagged = check_routing(idx, wts, idx_o, w_o, gap)
-    # outputs: a seeded sample of tokens (and every flagged one)
-    rng = np.random.default_rng(0)
-    sample = np.union1d(rng.choice(cfg.tokens, 192, replace=False), np.array(flagged, dtype=np.int64))
-    sample = np.union1d(sample, [0, cfg.tokens - 1])
-    err, l2, _ = check_layer(cfg, w, x, y, idx, wts, tokens=sample)
+    # outputs: every token
+    err, l2, _ = check_layer(cfg, w, x, y, idx, wts)
     print(f"prefill chunk 1024: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
 
 
@@ -232,42 +229,72 @@ def test_routing_copies_one_at_a_time(full):
     assert torch.equal(y1, y2)
 
 
-def test_stack_48_layers_first_three():
-    """48-layer stack, checked on its first 3 seeded layers: x_0 = x; layer l
-    reads bf16(RMSNorm(resid_l)); resid_{l+1} = resid_l + y_l (fp32 on the GPU).  Each
-    step is compared on 256 sampled tokens: the GPU's RMSNorm output against the
-    oracle's RMSNorm of the GPU residual, and the GPU layer against the oracle layer on
-    the GPU's own bf16 layer input.  Every layer applies the same code to its own
-    weights, so the first layers stand for the rest; the full 24 GB stack is the
-    bench's workload."""
+def test_stack_48_layers_against_oracle_stack():
+    """The 48-layer stack (the pages' model depth) at T = 1024, end to end: x_0 = x; layer l reads
+    bf16(RMSNorm(r_l)); r_{l+1} = r_l + y_l, the residual fp32 on the GPU and fp64 in the oracle.  The GPU runs all
+    1024 tokens through all 48 layers with no re-anchoring; the oracle stack carries 256 sampled tokens through
+    the same 48 layers from the same x.
+
+    Every routing decision the GPU takes in the stack is checked against the oracle's routing of the GPU's own
+    layer input (sets bit-exact except near-ties).  The two trajectories' layer inputs drift apart by the
+    accumulated rounding of earlier layers, so a token whose margin is below that drift may take a different set
+    on the two sides; there the oracle stack takes the GPU's set (counted and printed).  The final residuals
+    must agree within max|dr| / max|r| <= 1e-2; the drift of the bf16 layer input is printed every 8 layers."""
+    import math
+
     from bit_block_quantized_moe_b200 import moe_rmsnorm_residual
+    from gen import make_layer
 
     cfg = CONFIGS["stack"]
-    T, H = cfg.tokens, cfg.hidden
+    T, H, L, k = cfg.tokens, cfg.hidden, cfg.layers, cfg.top_k
+    assert L == 48
     rng = np.random.default_rng(3)
     sample = np.sort(rng.choice(T, 256, replace=False))
     x0 = make_x(cfg, seed=0)
     resid = torch.from_numpy(bf16_to_f32(x0)).cuda()
     xn = torch.empty((T, H), dtype=torch.int16, device="cuda")
     moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6)
-    for layer in range(3):
+    idx_g = np.empty((L, sample.size, k), dtype=np.int32)
+    w_g = np.empty((L, sample.size, k), dtype=np.float32)
+    xn_g = np.empty((L, sample.size, H), dtype=np.uint16)
+    for layer in range(L):
+        Lyr, _ = build_layer(cfg, layer=layer)
+        idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+        wts = torch.zeros((T, k), dtype=torch.float32, device="cuda")
+        y = Lyr.forward(xn, topk_idx=idx, topk_w=wts)
         torch.cuda.synchronize()
-        r_host = resid.cpu().numpy().astype(np.float64)
-        xn_host = xn.cpu().numpy().view(np.uint16)
-        want = oracle.rmsnorm(r_host[sample], 1e-6)
-        got = bf16_to_f32(xn_host[sample])
-        assert np.max(np.abs(got - want) / np.maximum(np.abs(want), 1e-3)) < 2 ** -8
-        L, w = build_layer(cfg, layer=layer)
-        idx = torch.full((T, cfg.top_k), -1, dtype=torch.int32, device="cuda")
-        wts = torch.zeros((T, cfg.top_k), dtype=torch.float32, device="cuda")
-        y = L.forward(xn, topk_idx=idx, topk_w=wts)
-        torch.cuda.synchronize()
-        L.check_status()
-        err, l2, flagged = check_layer(cfg, w, xn_host, bf16_to_f32(y.cpu().numpy().view(np.uint16)).astype(np.float64),
-                                       idx.cpu().numpy(), wts.cpu().numpy(), tokens=sample)
-        print(f"stack layer {layer}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
-        moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6)  # resid += y; next layer input
-        del L
+        Lyr.check_status()
+        xn_g[layer] = xn.cpu().numpy().view(np.uint16)[sample]
+        idx_g[layer] = idx.cpu().numpy()[sample]
+        w_g[layer] = wts.cpu().numpy()[sample]
+        moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6)  # r += y; the next layer's input
+        del Lyr
+    torch.cuda.synchronize()
+    r_gpu = resid.cpu().numpy()[sample].astype(np.float64)
+
+    r = None
+    followed, flagged = 0, 0
+    bounds = [0, 8, 16, 24, 32, 40, 47, 48]
+    for c0, c1 in zip(bounds[:-1], bounds[1:]):
+        lays = [make_layer(cfg, seed=0, layer=l) for l in range(c0, c1)]
+        # the layer input of layer c0 on both sides
+        u_o = bf16_to_f32(oracle.double_to_bf16(oracle.rmsnorm(bf16_to_f32(x0[sample]).astype(np.float64)
+                                                               if r is None else r, 1e-6)))
+        u_g = bf16_to_f32(xn_g[c0])
+        print(f"stack layer {c0:2d} input: max|du|/max|u| = {np.max(np.abs(u_g - u_o)) / np.max(np.abs(u_o)):.3e}")
+        for l, lay in zip(range(c0, c1), lays):  # every GPU routing decision, on the GPU's own layer input
+            idx_o, w_o, gap, _ = oracle.route(xn_g[l], lay["router_w"], lay["router_b"], k)
+            flagged += len(check_routing(idx_g[l], w_g[l], idx_o, w_o, gap))
+        r, _, _, nf, nm = oracle.stack(x0[sample], lays, k, cfg.inter, eps=1e-6, follow_idx=idx_g[c0:c1],
+                                       tie_gap=math.inf, resid_in=r)
+        followed += nf
+        del lays
+    err = np.max(np.abs(r_gpu - r)) / np.max(np.abs(r))
+    rel_l2 = np.linalg.norm(r_gpu - r) / np.linalg.norm(r)
+    print(f"stack of 48 layers, 256 tokens: final residual max|dr|/max|r| = {err:.3e}, relL2 {rel_l2:.3e}; "
+          f"near-tie routing differences on the GPU's own inputs: {flagged}; (layer, token) pairs where the two "
+          f"trajectories routed differently and the oracle took the GPU's set: {followed} of {L * sample.size}")
+    assert err <= 1e-2
 
 
 def test_prefill_chunk_32768(full):

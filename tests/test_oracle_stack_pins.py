@@ -191,3 +191,14 @@ def test_stack_follows_an_outside_routing_only_at_near_ties():
     r3, idx3, _, nf, nm = oracle.stack(x, lay, 2, 32, follow_idx=other, tie_gap=math.inf)
     assert nf == 3 * 4 and nm == 0 and np.array_equal(idx3, other)
     assert not np.array_equal(r3, r0)
+
+
+def test_stack_in_chunks_of_layers_equals_one_call():
+    cfg = MoeConfig("t", 64, 32, 8, 2, 4, "zipf")
+    lay = _layers(cfg, 5, seed=12)
+    x = make_x(4, 64, seed=12)
+    r, idx, gap, _, _ = oracle.stack(x, lay, 2, 32)
+    r2, idx2, gap2, _, _ = oracle.stack(x, lay[:2], 2, 32)
+    r3, idx3, gap3, _, _ = oracle.stack(x, lay[2:], 2, 32, resid_in=r2)
+    assert np.array_equal(r3, r) and np.array_equal(np.concatenate([idx2, idx3]), idx)
+    assert np.array_equal(np.concatenate([gap2, gap3]), gap)
