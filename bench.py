@@ -1,18 +1,23 @@
 #!/usr/bin/env python
 """Bench: one routed MoE layer over 2-bit (Q2) block-quantized experts on B200.
 
-Headline workload: the full-size decode/verify layer (hidden 2048, 512 routed
-experts, top-10 + 1 shared, intermediate 512, T = 3 tokens, uniform router).
-A step is one pass of the whole layer (router GEMV, top-k, dispatch, gate/up +
-SwiGLU, down, combine) over one batch of 3 synthetic tokens.  The same run
-also measures the 1024-token prefill chunk with the Zipf-skewed router and
-reports it under "prefill_t1024".
+Headline workload (the JSON line's `value`): the full-size decode/verify layer
+(hidden 2048, 512 routed experts, top-10 + 1 shared, intermediate 512, T = 3
+tokens, uniform router).  A step is one pass of the whole layer (router GEMV,
+top-k, gate/up + SwiGLU, down, combine) over one batch of 3 synthetic tokens.
+The same run measures, each in a block of its own:
+  decode_sweep   T = 1, 2, 3 on the four Zipf-routed layers of the 32768-token case;
+  prefill_t1024  the 1024-token prefill chunk with the Zipf-skewed router;
+  prefill_t32768 four layers at T = 32768 (one graph per step);
+  stack_t1024    48 layers with RMSNorm + residual between them at T = 1024
+                 (one graph per step over all 48 layers).
 
 Timing: steps are captured in CUDA graphs and timed with CUDA events on the
 launch stream, with a barrier + synchronize on both sides (max over ranks for
 N > 1).  Decode steps rotate over 24 distinct copies of the layer weights
-(11.8 GB) and 64 input slots, so a step never finds its weights in the 126 MB
-L2; a prefill step reads all 513 experts (> L2).
+(12 GB) and 64 input slots, so a step never finds its weights in the 126 MB
+L2; a prefill step reads all 513 experts (> L2).  SM clocks and throttle
+reasons are sampled through NVML every 10 ms while the timed regions run.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead (the
 reference arm of this benchmark; there is no runnable upstream code).
@@ -21,10 +26,10 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -37,16 +42,19 @@ EXPERT_BYTES = 983040          # one Q2 expert at hidden 2048 / intermediate 512
 SPEC_HBM_GBS = 8000.0          # headline HBM figure
 SPEC_BF16_TFLOPS = 2250.0      # dense bf16
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GAP_TIE = 1e-5                 # near-tie threshold on the k-th/(k+1)-th logit gap
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=24000)
-    ap.add_argument("--warmup", type=int, default=240)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill, 32768-token and stack blocks")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 48-layer stack block")
+    ap.add_argument("--no-32k", action="store_true", help="skip the 32768-token block and the decode sweep")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--prefill-steps", type=int, default=40)
     ap.add_argument("--decode-sets", type=int, default=24,
@@ -54,40 +62,50 @@ def parse():
     return ap.parse_args()
 
 
-# Sources the fused decode kernel is compiled from; an ncu summary under profiles/ records
-# their hash, and its DRAM traffic is reported only while the sources still match.
-# the files that make up the fused decode kernel's device code (kernels.cuh holds host declarations only)
+# ---------------------------------------------------------------------------
+# ncu summaries: DRAM traffic per launch is reported only while the kernel's sources still match the capture
+
+CSRC = os.path.join(ROOT, "bit_block_quantized_moe_b200", "csrc")
+# the files that make up each kernel's device code (kernels.cuh holds host declarations only)
 DECODE_SOURCES = ["decode.cu", "common.cuh", "sync.cuh", "router.cuh"]
+PREFILL_SOURCES = ["prefill.cu", "tc.cuh", "common.cuh", "sync.cuh"]
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_fused_kernel_t3.md")
+PREFILL_PROFILE = os.path.join(ROOT, "profiles", "tc_expert_kernel_prefill_t1024.md")
 
 
-def decode_source_hash() -> str:
-    import hashlib
-
+def source_hash(files) -> str:
     h = hashlib.sha256()
-    for f in DECODE_SOURCES:
-        with open(os.path.join(ROOT, "bit_block_quantized_moe_b200", "csrc", f), "rb") as fh:
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_decode_traffic():
-    """(bytes per launch, note) from the committed ncu summary if it was taken on these sources, else (None, why)."""
+def decode_source_hash() -> str:
+    return source_hash(DECODE_SOURCES)
+
+
+def prefill_source_hash() -> str:
+    return source_hash(PREFILL_SOURCES)
+
+
+def profiled_traffic(path, files, key="dram bytes per launch"):
+    """(bytes per launch, note) from a committed ncu summary if it was taken on these sources, else (None, why)."""
     try:
-        text = open(DECODE_PROFILE).read()
+        text = open(path).read()
     except OSError:
         return None, "no ncu summary"
     src = traffic = None
     for line in text.splitlines():
         if line.startswith("sources sha256:"):
             src = line.split(":", 1)[1].strip()
-        if line.startswith("dram bytes per launch:"):
+        if line.startswith(key + ":"):
             traffic = float(line.split(":", 1)[1].strip())
     if src is None or traffic is None:
         return None, "summary lacks hash or traffic"
-    if src != decode_source_hash():
+    if src != source_hash(files):
         return None, "kernel changed since the ncu capture"
-    return traffic, "ncu dram__bytes_read.sum + dram__bytes_write.sum, " + os.path.basename(DECODE_PROFILE)
+    return traffic, "ncu dram__bytes_read.sum + dram__bytes_write.sum, " + os.path.basename(path)
 
 
 def load_peaks():
@@ -100,59 +118,92 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# clocks sampled during the timed region
+# clocks sampled during the timed regions (NVML, every 10 ms)
 
 
 class ClockSampler:
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
-        self.proc = None
-        self.lines = []
+    """Samples SM clock and clock-event reasons of one GPU in a thread; timed regions are marked with
+    window(), and the summary covers the samples taken inside them."""
 
-    def __enter__(self):
-        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-             "clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, uuid: str, period_s: float = 0.01):
+        self.samples = []  # (t, sm_mhz, max_mhz, reasons mask)
+        self.windows = []
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self._reasons = get
+            self.ok = True
+        except Exception as e:  # no NVML: the line says so
+            self.err = str(e)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.thread.join(timeout=2)
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = self._reasons(h)
+                self.samples.append((time.perf_counter(), sm, self.max_mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self.th.join(timeout=2)
+
+    class _Win:
+        def __init__(self, s, name):
+            self.s, self.name = s, name
+
+        def __enter__(self):
+            self.t0 = time.perf_counter()
+            return self
+
+        def __exit__(self, *a):
+            self.s.windows.append((self.name, self.t0, time.perf_counter()))
+
+    def window(self, name):
+        return ClockSampler._Win(self, name)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvml unavailable"}
+        inside = [s for s in self.samples if any(t0 <= s[0] <= t1 for _, t0, t1 in self.windows)]
+        sm = [s[1] for s in inside]
+        mask = 0
+        for s in inside:
+            mask |= s[3]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(v for k, v in self.REASONS.items() if mask & k), "samples": len(sm),
+                "window_s": round(sum(t1 - t0 for _, t0, t1 in self.windows), 3),
+                "windows": sorted({n for n, _, _ in self.windows}), "source": "nvml, 10 ms"}
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
 
 
 # ---------------------------------------------------------------------------
@@ -186,44 +237,20 @@ def barrier(world: int):
 
 
 # ---------------------------------------------------------------------------
-# our arm
+# timing
 
 
-def make_layer_sets(cfg, n_distinct: int, n_sets: int, seed: int, device):
-    """n_sets device copies of n_distinct seeded layers (distinct memory -> no L2 reuse)."""
-    import torch
-
-    from bit_block_quantized_moe_b200 import Q2MoeLayer
-    from gen import make_layer
-
-    base = []
-    for l in range(n_distinct):
-        w = make_layer(cfg, seed=seed, layer=l)
-        base.append(Q2MoeLayer(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, w["router_w"], w["router_b"],
-                               w["experts"], w["shared"], device=device))
-    sets = []
-    for i in range(n_sets):
-        b = base[i % n_distinct]
-        if i < n_distinct:
-            sets.append((b.router_w, b.router_b, b.experts, b.shared))
-        else:
-            sets.append((b.router_w.clone(), None if b.router_b is None else b.router_b.clone(), b.experts.clone(),
-                         b.shared.clone()))
-    torch.cuda.synchronize()
-    return base[0].dims, sets
-
-
-def capture(fn, n_steps, stream):
+def capture(fn, n_steps, stream, first=0):
     import torch
 
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
-        for i in range(n_steps):
+        for i in range(first, first + n_steps):
             fn(i)
     return g
 
 
-def time_graph_steps(fn, K, W, stream, world, chunk=240, sampler=None):
+def time_graph_steps(fn, K, W, stream, world, chunk=240, win=None):
     """Warm up W steps, then time exactly K steps (graphs of <= chunk steps); returns seconds (max over ranks)."""
     import torch
 
@@ -243,8 +270,7 @@ def time_graph_steps(fn, K, W, stream, world, chunk=240, sampler=None):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    ctx = sampler if sampler is not None else _Null()
-    with ctx, torch.cuda.stream(stream):
+    with (win if win is not None else _Null()), torch.cuda.stream(stream):
         start.record(stream)
         for _ in range(full):
             g_full.replay()
@@ -259,17 +285,24 @@ def time_graph_steps(fn, K, W, stream, world, chunk=240, sampler=None):
     return max_over_ranks(secs, world)
 
 
-class _Null:
-    def __enter__(self):
-        return self
+def soak(fn, seconds, stream, win):
+    """Replays the step for about `seconds` (untimed), so that the clock sampler sees the workload's clocks."""
+    import torch
 
-    def __exit__(self, *a):
-        return False
+    g = capture(fn, 240, stream)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with win, torch.cuda.stream(stream):
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(20):
+                g.replay()
+            torch.cuda.synchronize()
+    del g
 
 
 def traced_kernel_ms(fn, n_steps, kernel_id, stream):
-    """Average duration of one library kernel over n_steps graph-captured steps,
-    from CUDA events the library records around that kernel."""
+    """Average duration of one library kernel over n_steps graph-captured steps, from CUDA events the library
+    records around that kernel on the launch stream."""
     import torch
 
     import bit_block_quantized_moe_b200 as M
@@ -299,112 +332,184 @@ def traced_kernel_ms(fn, n_steps, kernel_id, stream):
 def gpu_uuid(dev):
     import torch
 
-    try:
-        u = str(torch.cuda.get_device_properties(dev).uuid)
-        return u if u.startswith("GPU-") else "GPU-" + u
-    except Exception:
-        return str(dev)
+    u = str(torch.cuda.get_device_properties(dev).uuid)
+    return u if u.startswith("GPU-") else "GPU-" + u
 
 
-def run_ours(args, world, rank, local):
+def layer_bytes(touched, E, H, T):
+    """Algorithmic bytes of one layer step: touched experts + shared, the router, x in and out."""
+    return (touched + 1) * EXPERT_BYTES + E * H * 4 + 2 * T * H * 2
+
+
+def layer_flops(T, k, H, I, E):
+    return T * (k + 1) * 6 * H * I + 2 * T * H * E
+
+
+def routing_check(x_bits, router_w, router_b, idx_gpu, top_k):
+    """The oracle's routing of the same tokens: near ties (k-th/(k+1)-th gap < 1e-5) and set differences."""
+    import numpy as np
+
+    import oracle
+
+    idx_o, _, gap, _ = oracle.route(x_bits, router_w, router_b, top_k)
+    differ = np.array([set(a) != set(b) for a, b in zip(idx_gpu.tolist(), idx_o.tolist())])
+    ties = gap < GAP_TIE
+    return {"tokens": int(len(gap)), "near_ties": int(ties.sum()), "sets_differ": int(differ.sum()),
+            "sets_differ_beyond_near_ties": int((differ & ~ties).sum())}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+
+def make_layer_sets(cfg, n_distinct: int, n_sets: int, seed: int, device, on_device=False, first_layer=0):
+    """n_sets device copies of n_distinct seeded layers (distinct memory -> no L2 reuse); also the host router
+    weights of the distinct layers (for the oracle's routing check)."""
+    import torch
+
+    from bit_block_quantized_moe_b200 import Q2MoeLayer
+    from gen import make_layer
+    from gen.moe_inputs import make_layer_device
+
+    base, routers = [], []
+    for l in range(first_layer, first_layer + n_distinct):
+        w = make_layer_device(cfg, seed, l, device) if on_device else make_layer(cfg, seed=seed, layer=l)
+        base.append(Q2MoeLayer(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k, w["router_w"], w["router_b"],
+                               w["experts"], w["shared"], device=device))
+        routers.append((base[-1].router_w.cpu().numpy(),
+                        None if base[-1].router_b is None else base[-1].router_b.cpu().numpy()))
+        del w
+    sets = []
+    for i in range(n_sets):
+        b = base[i % n_distinct]
+        if i < n_distinct:
+            sets.append((b.router_w, b.router_b, b.experts, b.shared))
+        else:
+            sets.append((b.router_w.clone(), None if b.router_b is None else b.router_b.clone(), b.experts.clone(),
+                         b.shared.clone()))
+    torch.cuda.synchronize()
+    return base[0].dims, sets, routers
+
+
+def run_decode(args, cfg, sets, routers, dims, T, K, W, world, rank, dev, stream, peaks, peak_src, sampler,
+               with_e2e=False):
+    """Decode steps of T tokens rotating over the weight sets and 64 input slots."""
     import numpy as np
     import torch
 
     import bit_block_quantized_moe_b200 as M
-    from gen import CONFIGS, make_x
+    from gen import make_x
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    peaks, peak_src = load_peaks()
-    stream = torch.cuda.Stream()
-    K, W = args.steps, max(args.warmup, 3)
-
-    # ---- decode layer, T = 3 -------------------------------------------------------
-    cfg = CONFIGS["decode"]
-    T, H = cfg.tokens, cfg.hidden
-    n_sets, n_slots = args.decode_sets, 64
-    dims, sets = make_layer_sets(cfg, min(4, n_sets), n_sets, args.seed, dev)
-    xs = torch.stack([torch.from_numpy(make_x(T, H, seed=1000 * (rank + 1) + s).view(np.int16)) for s in range(n_slots)])
-    xs = xs.to(dev)
+    H = cfg.hidden
+    n_sets, n_slots = len(sets), 64
+    n_distinct = len(routers)
+    xs_np = [make_x(T, H, seed=1000 * (rank + 1) + 100 * T + s) for s in range(n_slots)]
+    xs = torch.stack([torch.from_numpy(x.view(np.int16)) for x in xs_np]).to(dev)
     outs = torch.empty_like(xs)
     ws = torch.zeros(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
-    idx_all = torch.empty((n_sets * n_slots, T, cfg.top_k), dtype=torch.int32, device=dev)
-    w_all = torch.empty((n_sets * n_slots, T, cfg.top_k), dtype=torch.float32, device=dev)
+    idx_all = torch.empty((n_distinct * n_slots, T, cfg.top_k), dtype=torch.int32, device=dev)
+    w_all = torch.empty((n_distinct * n_slots, T, cfg.top_k), dtype=torch.float32, device=dev)
 
     def step(i):
         rw, rb, ex, sh = sets[i % n_sets]
         s = i % n_slots
         M.moe_layer_forward(dims, xs[s], rw, rb, ex, sh, outs[s], T, ws, stream=stream)
 
-    # routing of every (set, slot) pair for the algorithmic-byte count
+    # routing of every (distinct layer, slot) pair: touched experts for the byte count, and the oracle's check
     with torch.cuda.stream(stream):
-        for si in range(n_sets):
+        for si in range(n_distinct):
+            rw, rb, ex, sh = sets[si]
             for s in range(n_slots):
-                rw, rb, ex, sh = sets[si]
                 M.moe_route(dims, xs[s], rw, rb, T, idx_all[si * n_slots + s], w_all[si * n_slots + s], ws,
                             stream=stream)
     torch.cuda.synchronize()
     idx_np = idx_all.cpu().numpy()
-    touched = np.array([len(np.unique(idx_np[p])) for p in range(n_sets * n_slots)])
+    touched = np.array([len(np.unique(idx_np[p])) for p in range(n_distinct * n_slots)])
+    check = None
+    if rank == 0:
+        ci = [routing_check(np.concatenate(xs_np), routers[si][0], routers[si][1],
+                            idx_np[si * n_slots:(si + 1) * n_slots].reshape(-1, cfg.top_k), cfg.top_k)
+              for si in range(n_distinct)]
+        check = {k: sum(c[k] for c in ci) for k in ci[0]}
 
-    def step_pair(i):
-        return (i % n_sets) * n_slots + (i % n_slots)
-
-    sampler = ClockSampler(gpu_uuid(dev)) if rank == 0 else None
-    secs = time_graph_steps(step, K, W, stream, world, sampler=sampler)
+    win = sampler.window(f"decode T={T}") if sampler is not None else None
+    secs = time_graph_steps(step, K, W, stream, world, win=win)
     ms_per_step = secs * 1e3 / K
-    value = world * T * K / secs
+    avg_touched = float(np.mean([touched[(i % n_sets % n_distinct) * n_slots + (i % n_slots)] for i in range(K)]))
+    bytes_ = layer_bytes(avg_touched, cfg.n_experts, H, T)
+    out = {"T": T, "ms_per_step": ms_per_step, "value": world * T * K / secs, "unit": "tokens/s", "steps": K,
+           "touched_experts_per_step": avg_touched, "bytes_per_step": bytes_,
+           "achieved_gbs": bytes_ / (ms_per_step * 1e-3) / 1e9,
+           "frac_of_measured_hbm": bytes_ / (ms_per_step * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+           "frac_of_8tbs": bytes_ / (ms_per_step * 1e-3) / 1e9 / SPEC_HBM_GBS, "routing_check": check}
+    if sampler is not None and T == 3:
+        soak(step, 1.0, stream, sampler.window("decode T=3 soak"))
 
-    avg_touched = float(np.mean([touched[step_pair(i)] for i in range(min(K, 24 * 64 * 4))]))
-    expert_bytes = (avg_touched + 1) * EXPERT_BYTES
-    layer_bytes = expert_bytes + cfg.n_experts * H * 4 + 2 * T * H * 2
-    # dominant kernel: the fused decode kernel (the whole layer in one launch)
-    n_trace = min(240, max(24, K))
-    kern_ms = traced_kernel_ms(step, n_trace, M.MOE_KERNEL["decode_fused"], stream)
-    hbm_peak = float(peaks["hbm_gbs"])
-    kern_gbs = layer_bytes / (kern_ms * 1e-3) / 1e9
-    traffic, traffic_note = profiled_decode_traffic()
-    layer_gbs = layer_bytes / (ms_per_step * 1e-3) / 1e9
-
-    # ---- end to end through the public API, host buffers --------------------------------
-    n_e2e = min(K, 2000)
-    xh = torch.empty((n_slots, T, H), dtype=torch.int16).pin_memory()
-    xh.copy_(xs.cpu())
-    oh = torch.empty((n_slots, T, H), dtype=torch.int16).pin_memory()
-    xd = torch.empty((T, H), dtype=torch.int16, device=dev)
-    od = torch.empty((T, H), dtype=torch.int16, device=dev)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            xd.copy_(xh[i], non_blocking=True)
-            rw, rb, ex, sh = sets[i % n_sets]
-            M.moe_layer_forward(dims, xd, rw, rb, ex, sh, od, T, ws, stream=stream)
-            oh[i].copy_(od, non_blocking=True)
+    if with_e2e:
+        # end to end through the public API, host buffers copied in and out every step
+        n_e2e = min(K, 2000)
+        xh = torch.empty((n_slots, T, H), dtype=torch.int16).pin_memory()
+        xh.copy_(xs.cpu())
+        oh = torch.empty((n_slots, T, H), dtype=torch.int16).pin_memory()
+        xd = torch.empty((T, H), dtype=torch.int16, device=dev)
+        od = torch.empty((T, H), dtype=torch.int16, device=dev)
         torch.cuda.synchronize()
-        e0.record(stream)
-        for i in range(n_e2e):
-            s = i % n_slots
-            xd.copy_(xh[s], non_blocking=True)
-            rw, rb, ex, sh = sets[i % n_sets]
-            M.moe_layer_forward(dims, xd, rw, rb, ex, sh, od, T, ws, stream=stream)
-            oh[s].copy_(od, non_blocking=True)
-        e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
-    e2e_value = world * T * n_e2e / e2e_secs
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                xd.copy_(xh[i], non_blocking=True)
+                rw, rb, ex, sh = sets[i % n_sets]
+                M.moe_layer_forward(dims, xd, rw, rb, ex, sh, od, T, ws, stream=stream)
+                oh[i].copy_(od, non_blocking=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(n_e2e):
+                s = i % n_slots
+                xd.copy_(xh[s], non_blocking=True)
+                rw, rb, ex, sh = sets[i % n_sets]
+                M.moe_layer_forward(dims, xd, rw, rb, ex, sh, od, T, ws, stream=stream)
+                oh[s].copy_(od, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_secs = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+        out["e2e"] = {"value": world * T * n_e2e / e2e_secs, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+                      "d2h_bytes_per_step": T * H * 2, "steps": n_e2e}
     M.moe_check_status(ws)
+    return out
 
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from gen import CONFIGS
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream()
+    K, W = args.steps, max(args.warmup, 3)
+    sampler = ClockSampler(gpu_uuid(dev)).start() if rank == 0 else None
+    hbm_peak = float(peaks["hbm_gbs"])
+
+    # ---- headline: decode layer, T = 3, uniform router ------------------------------------------------
+    cfg = CONFIGS["decode"]
+    T = cfg.tokens
+    n_distinct = min(4, args.decode_sets)
+    dims, sets, routers = make_layer_sets(cfg, n_distinct, args.decode_sets, args.seed, dev)
+    d = run_decode(args, cfg, sets, routers, dims, T, K, W, world, rank, dev, stream, peaks, peak_src, sampler,
+                   with_e2e=True)
+    del sets
+    traffic, traffic_note = profiled_traffic(DECODE_PROFILE, DECODE_SOURCES)
     result = {
         "metric": METRIC,
-        "value": value,
+        "value": d["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
         "warmup": W,
-        "ms_per_step": ms_per_step,
+        "ms_per_step": d["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -416,43 +521,46 @@ def run_ours(args, world, rank, local):
             "global_batch": T * world,
             "seq_len": T,
             "parallelism": f"{world} independent token-parallel replicas, no collective",
-            "l2": f"{n_sets} rotating weight copies ({n_sets * 0.504:.1f} GB) and 64 input slots: inputs larger "
-                  "than L2",
-            "touched_experts_per_step": avg_touched,
+            "l2": f"{args.decode_sets} rotating weight copies ({args.decode_sets * 0.504:.1f} GB) and 64 input slots: "
+                  "inputs larger than L2",
+            "touched_experts_per_step": d["touched_experts_per_step"],
         },
+        # The fused decode kernel is the whole step (one launch per step, nothing else in the timed region), so
+        # its average launch duration is the timed region's event time divided by the steps.
         "roofline": {
             "bound": "hbm",
             "kernel": "decode_fused_kernel (router, top-k, gate/up + SwiGLU, down, combine)",
-            "achieved": kern_gbs,
+            "achieved": d["achieved_gbs"],
             "peak": hbm_peak,
             "unit": "GB/s",
-            "frac": kern_gbs / hbm_peak,
+            "frac": d["achieved_gbs"] / hbm_peak,
             "traffic": traffic,
             "traffic_source": traffic_note,
             "peak_source": f"{peak_src} hbm_gbs",
-            "kernel_ms": kern_ms,
-            "algorithmic_bytes": layer_bytes,
+            "kernel_ms": d["ms_per_step"],
+            "kernel_ms_source": "CUDA events on the launch stream over the timed region / steps (1 launch per step)",
+            "algorithmic_bytes": d["bytes_per_step"],
+            "frac_of_8tbs": d["frac_of_8tbs"],
         },
-        "layer_roofline": {
-            "bytes_per_step": layer_bytes,
-            "achieved_gbs": layer_gbs,
-            "frac_of_measured": layer_gbs / hbm_peak,
-            "frac_of_8tbs": layer_gbs / SPEC_HBM_GBS,
-        },
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
-                "d2h_bytes_per_step": T * H * 2, "steps": n_e2e},
-        "gpu_launches": 1 * K,
+        "routing_check": d["routing_check"],
+        "e2e": d["e2e"],
+        "gpu_launches": K,
     }
-    if sampler is not None:
-        result["clocks"] = sampler.summary()
 
-    # ---- prefill chunk, T = 1024 ---------------------------------------------------------
     if not args.no_prefill:
-        result["prefill_t1024"] = run_prefill(args, world, rank, dev, stream, peaks, peak_src)
+        result["prefill_t1024"] = run_prefill(args, world, rank, dev, stream, peaks, peak_src, sampler)
+        if not args.no_32k:
+            result["prefill_t32768"], result["decode_sweep"] = run_32k(args, world, rank, dev, stream, peaks,
+                                                                       peak_src, sampler, K, W)
+        if not args.no_stack:
+            result["stack_t1024"] = run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler)
+    if sampler is not None:
+        sampler.stop()
+        result["clocks"] = sampler.summary()
     return result
 
 
-def run_prefill(args, world, rank, dev, stream, peaks, peak_src):
+def run_prefill(args, world, rank, dev, stream, peaks, peak_src, sampler):
     import numpy as np
     import torch
 
@@ -461,11 +569,11 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src):
 
     cfg = CONFIGS["prefill"]
     T, H = cfg.tokens, cfg.hidden
-    dims, sets = make_layer_sets(cfg, 1, 1, args.seed, dev)
+    dims, sets, routers = make_layer_sets(cfg, 1, 1, args.seed, dev)
     rw, rb, ex, sh = sets[0]
     n_slots = 4
-    xs = torch.stack([torch.from_numpy(make_x(T, H, seed=2000 * (rank + 1) + s).view(np.int16))
-                      for s in range(n_slots)]).to(dev)
+    xs_np = [make_x(T, H, seed=2000 * (rank + 1) + s) for s in range(n_slots)]
+    xs = torch.stack([torch.from_numpy(x.view(np.int16)) for x in xs_np]).to(dev)
     outs = torch.empty_like(xs)
     ws = torch.zeros(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
     idx = torch.empty((n_slots, T, cfg.top_k), dtype=torch.int32, device=dev)
@@ -479,18 +587,26 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src):
         for s in range(n_slots):
             M.moe_route(dims, xs[s], rw, rb, T, idx[s], wts[s], ws, stream=stream)
     torch.cuda.synchronize()
-    touched = float(np.mean([len(np.unique(idx[s].cpu().numpy())) for s in range(n_slots)]))
+    idx_np = idx.cpu().numpy()
+    touched = float(np.mean([len(np.unique(idx_np[s])) for s in range(n_slots)]))
+    check = routing_check(xs_np[0], routers[0][0], routers[0][1], idx_np[0], cfg.top_k) if rank == 0 else None
     K = args.prefill_steps
-    secs = time_graph_steps(step, K, 3, stream, world, chunk=20)
+    win = sampler.window("prefill T=1024") if sampler is not None else None
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=20, win=win)
     ms = secs * 1e3 / K
-    bytes_ = (touched + 1) * EXPERT_BYTES + cfg.n_experts * H * 4 + 2 * T * H * 2
-    flops = T * (cfg.top_k + 1) * 6 * H * cfg.inter + 2 * T * H * cfg.n_experts
+    bytes_ = layer_bytes(touched, cfg.n_experts, H, T)
+    flops = layer_flops(T, cfg.top_k, H, cfg.inter, cfg.n_experts)
     hbm = float(peaks["hbm_gbs"])
     tflops = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     t_roof = max(bytes_ / (hbm * 1e9), flops / (tflops * 1e12))
     t_roof_spec = max(bytes_ / (SPEC_HBM_GBS * 1e9), flops / (SPEC_BF16_TFLOPS * 1e12))
+    # the dominant kernel: gate/up + SwiGLU (tcgen05), timed by events the library records around it
     gu_ms = traced_kernel_ms(step, min(K, 8), M.MOE_KERNEL["gate_up"], stream)
+    dn_ms = traced_kernel_ms(step, min(K, 8), M.MOE_KERNEL["down"], stream)
     gu_flops = (T * cfg.top_k + T) * 4 * H * cfg.inter
+    gu_bytes = (touched + 1) * EXPERT_BYTES * 2 / 3 + (T * cfg.top_k + T) * H * 2  # gate/up sections + token rows
+    traffic, traffic_note = profiled_traffic(PREFILL_PROFILE, PREFILL_SOURCES, "dram bytes per launch (gate/up)")
+    M.moe_check_status(ws)
     return {
         "value": world * T * K / secs,
         "unit": "tokens/s",
@@ -503,9 +619,140 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src):
         "binding": "hbm" if bytes_ / (hbm * 1e9) >= flops / (tflops * 1e12) else "tensor",
         "roofline_frac_of_measured": t_roof / (ms * 1e-3),
         "roofline_frac_of_spec": t_roof_spec / (ms * 1e-3),
-        "gate_up_kernel_ms": gu_ms,
-        "gate_up_tflops": gu_flops / (gu_ms * 1e-3) / 1e12,
         "peak_source": peak_src,
+        "routing_check": check,
+        "roofline": {"bound": "hbm", "kernel": "tc_expert_kernel<0> (gate/up + SwiGLU, tcgen05)",
+                     "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": gu_bytes / (gu_ms * 1e-3) / 1e9 / hbm, "traffic": traffic,
+                     "traffic_source": traffic_note, "kernel_ms": gu_ms, "algorithmic_bytes": gu_bytes,
+                     "tflops": gu_flops / (gu_ms * 1e-3) / 1e12},
+        "down_kernel_ms": dn_ms,
+    }
+
+
+def run_32k(args, world, rank, dev, stream, peaks, peak_src, sampler, K_dec, W_dec):
+    """Four Zipf-routed layers at T = 32768 (one graph per step over the four layers), then the decode sweep
+    T = 1, 2, 3 on 24 rotating copies of the same four layers."""
+    import numpy as np
+    import torch
+
+    import bit_block_quantized_moe_b200 as M
+    from gen import CONFIGS, make_x
+
+    cfg = CONFIGS["prefill_32k"]
+    T, H, L = cfg.tokens, cfg.hidden, cfg.layers
+    dims, sets, routers = make_layer_sets(cfg, L, args.decode_sets, args.seed, dev, on_device=True)
+    x = torch.from_numpy(make_x(T, H, seed=3000 + rank).view(np.int16)).to(dev)
+    outs = torch.empty((L, T, H), dtype=torch.int16, device=dev)
+    ws = torch.zeros(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
+    idx = torch.empty((L, T, cfg.top_k), dtype=torch.int32, device=dev)
+    wts = torch.empty((L, T, cfg.top_k), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for l in range(L):
+            rw, rb, ex, sh = sets[l]
+            M.moe_route(dims, x, rw, rb, T, idx[l], wts[l], ws, stream=stream)
+    torch.cuda.synchronize()
+    idx_np = idx.cpu().numpy()
+    touched = [len(np.unique(idx_np[l])) for l in range(L)]
+
+    def step(i):
+        for l in range(L):
+            rw, rb, ex, sh = sets[l]
+            M.moe_layer_forward(dims, x, rw, rb, ex, sh, outs[l], T, ws, stream=stream)
+
+    K = 4
+    win = sampler.window("prefill T=32768") if sampler is not None else None
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=K, win=win)
+    ms_layer = secs * 1e3 / (K * L)
+    bytes_ = sum(layer_bytes(t, cfg.n_experts, H, T) for t in touched) / L
+    flops = layer_flops(T, cfg.top_k, H, cfg.inter, cfg.n_experts)
+    hbm = float(peaks["hbm_gbs"])
+    tflops = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    t_roof = max(bytes_ / (hbm * 1e9), flops / (tflops * 1e12))
+    M.moe_check_status(ws)
+    big = {
+        "value": world * T * K * L / secs, "unit": "tokens/s (layer passes)", "ms_per_layer": ms_layer,
+        "ms_per_step": ms_layer * L, "layers_per_step": L, "steps": K,
+        "workload": "4 full-size layers (hidden 2048, 512 experts top-10 + shared, inter 512), T=32768, Zipf router; "
+                    "each layer reads the same x",
+        "bytes_per_layer": bytes_, "flops_per_layer": flops,
+        "binding": "hbm" if bytes_ / (hbm * 1e9) >= flops / (tflops * 1e12) else "tensor",
+        "roofline_frac_of_measured": t_roof / (ms_layer * 1e-3), "peak_source": peak_src,
+    }
+    del ws, outs, idx, wts
+    torch.cuda.empty_cache()
+    sweep = {}
+    for Td in (1, 2, 3):
+        r = run_decode(args, cfg, sets, routers, dims, Td, min(K_dec, 2000), W_dec, world, rank, dev, stream, peaks,
+                       peak_src, sampler)
+        sweep[f"T{Td}"] = {k: r[k] for k in ("value", "unit", "ms_per_step", "touched_experts_per_step",
+                                             "bytes_per_step", "achieved_gbs", "frac_of_measured_hbm",
+                                             "frac_of_8tbs", "routing_check")}
+    sweep["workload"] = "decode T=1,2,3 on 24 rotating copies of the four Zipf-routed 32768-token-case layers"
+    del sets
+    torch.cuda.empty_cache()
+    return big, sweep
+
+
+def run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler):
+    """48 full-size layers, T = 1024: x_0 = x; layer l reads bf16(RMSNorm(r_l)); r_{l+1} = r_l + y_l.  One CUDA
+    graph per step over all 48 layers (the residual reset to x first)."""
+    import numpy as np
+    import torch
+
+    import bit_block_quantized_moe_b200 as M
+    from gen import CONFIGS, make_x
+
+    cfg = CONFIGS["stack"]
+    T, H, L = cfg.tokens, cfg.hidden, cfg.layers
+    dims, sets, routers = make_layer_sets(cfg, L, L, args.seed, dev, on_device=True)
+    x = torch.from_numpy((make_x(T, H, seed=4000 + rank).astype(np.uint32) << 16).view(np.float32)).to(dev)
+    resid = torch.empty_like(x)
+    xn = torch.empty((T, H), dtype=torch.int16, device=dev)
+    y = torch.empty((T, H), dtype=torch.int16, device=dev)
+    ws = torch.zeros(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
+    idx = torch.empty((T, cfg.top_k), dtype=torch.int32, device=dev)
+
+    def step(i):
+        resid.copy_(x)
+        M.moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6, stream=stream)
+        for l in range(L):
+            rw, rb, ex, sh = sets[l]
+            M.moe_layer_forward(dims, xn, rw, rb, ex, sh, y, T, ws, stream=stream)
+            M.moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6, stream=stream)
+
+    # touched experts per layer on the stack's own layer inputs (one eager pass)
+    touched = []
+    with torch.cuda.stream(stream):
+        resid.copy_(x)
+        M.moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6, stream=stream)
+        for l in range(L):
+            rw, rb, ex, sh = sets[l]
+            M.moe_layer_forward(dims, xn, rw, rb, ex, sh, y, T, ws, topk_idx_out=idx, stream=stream)
+            touched.append(len(np.unique(idx.cpu().numpy())))
+            M.moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6, stream=stream)
+    torch.cuda.synchronize()
+    K = max(1, min(args.steps, 5))
+    win = sampler.window("stack 48 x T=1024") if sampler is not None else None
+    with torch.cuda.stream(stream):
+        secs = time_graph_steps(step, K, 3, stream, world, chunk=1, win=win)
+    ms = secs * 1e3 / K
+    bytes_ = sum(layer_bytes(t, cfg.n_experts, H, T) for t in touched)
+    flops = L * layer_flops(T, cfg.top_k, H, cfg.inter, cfg.n_experts)
+    hbm = float(peaks["hbm_gbs"])
+    tflops = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    t_roof = max(bytes_ / (hbm * 1e9), flops / (tflops * 1e12))
+    M.moe_check_status(ws)
+    del sets
+    torch.cuda.empty_cache()
+    return {
+        "value": world * T * K / secs, "unit": "tokens/s (through all 48 layers)", "ms_per_step": ms,
+        "ms_per_layer": ms / L, "steps": K, "layers": L,
+        "workload": "48 full-size layers (hidden 2048, 512 experts top-10 + shared, inter 512), T=1024, Zipf router, "
+                    "RMSNorm eps 1e-6 + residual between layers, independent seeded weights per layer (24 GB)",
+        "touched_experts_mean": float(np.mean(touched)), "bytes_per_step": bytes_, "flops_per_step": flops,
+        "roofline_frac_of_measured": t_roof / (ms * 1e-3), "peak_source": peak_src,
+        "launches_per_layer": 12,
     }
 
 
@@ -513,15 +760,14 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src):
 # CPU oracle legs
 
 
-def oracle_decode_tokens_per_s(budget_s: float, seed: int, max_tokens=4096):
+def oracle_decode_tokens_per_s(budget_s: float, seed: int, threads: int, max_tokens=4096):
     """Time the fp64 oracle on decode-layer tokens (hidden 2048, 512 experts top-10) for about budget_s seconds."""
-    import numpy as np
-
     import oracle
     from gen import CONFIGS, make_layer, make_x
 
     cfg = CONFIGS["decode"]
     w = make_layer(cfg, seed=seed, layer=0)
+    oracle.set_num_threads(threads)
     nthr = oracle.num_threads()
     batch = max(3, nthr)
     done, t_used, i = 0, 0.0, 0
@@ -532,14 +778,13 @@ def oracle_decode_tokens_per_s(budget_s: float, seed: int, max_tokens=4096):
         t_used += time.perf_counter() - t0
         done += batch
         i += 1
+    oracle.set_num_threads(0)
     return done / t_used, nthr, done, t_used
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    import numpy as np
-
     import oracle
     from gen import CONFIGS, make_layer, make_x
 
@@ -611,10 +856,13 @@ def main():
     __graft_entry__.build()
     res = run_ours(args, world, rank, local)
     if rank == 0 and not args.no_cpu:
-        tps, nthr, ntok, tsec = oracle_decode_tokens_per_s(12.0, args.seed)
+        tps, nthr, ntok, tsec = oracle_decode_tokens_per_s(10.0, args.seed, 0)
+        tps1, _, ntok1, tsec1 = oracle_decode_tokens_per_s(6.0, args.seed, 1, max_tokens=64)
         res["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthr, "kind": "oracle",
                                "sample": f"{ntok} decode-layer tokens (hidden 2048, 512 experts top-10) in {tsec:.1f} s, "
-                                         f"OpenMP over tokens"}
+                                         f"OpenMP over tokens",
+                               "one_core": {"value": tps1, "unit": "tokens/s", "cores": 1,
+                                            "sample": f"{ntok1} tokens in {tsec1:.1f} s"}}
     if world > 1:
         import torch.distributed as dist
 

@@ -19,9 +19,8 @@ class Q2MoeLayer:
                  shared_canon, device="cuda", max_tokens: int = 0):
         self.dims = B.moe_dims(hidden, inter, n_experts, top_k)
         self.device = torch.device(device)
-        self.router_w = torch.as_tensor(np.ascontiguousarray(router_w, dtype=np.float32)).to(self.device)
-        self.router_b = None if router_b is None else torch.as_tensor(
-            np.ascontiguousarray(router_b, dtype=np.float32)).to(self.device)
+        self.router_w = self._f32(router_w)
+        self.router_b = None if router_b is None else self._f32(router_b)
         pe = B.moe_packed_expert_bytes(self.dims)
         ce = B.moe_canonical_expert_bytes(self.dims)
         if pe == 0 or ce == 0:
@@ -35,8 +34,17 @@ class Q2MoeLayer:
         if max_tokens:
             self.reserve(max_tokens)
 
+    def _f32(self, a):
+        if isinstance(a, torch.Tensor):
+            return a.detach().to(self.device, torch.float32).contiguous()
+        return torch.as_tensor(np.ascontiguousarray(a, dtype=np.float32)).to(self.device)
+
     def _pack(self, canon, n, ce, dst):
-        src = torch.as_tensor(np.ascontiguousarray(canon, dtype=np.uint8).reshape(-1))
+        if isinstance(canon, torch.Tensor):
+            src = canon.detach().reshape(-1)
+            assert src.dtype == torch.uint8
+        else:
+            src = torch.as_tensor(np.ascontiguousarray(canon, dtype=np.uint8).reshape(-1))
         assert src.numel() == n * ce
         # pack in slices to bound the temporary device copy
         per = max(1, (256 << 20) // ce)

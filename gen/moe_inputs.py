@@ -143,3 +143,37 @@ def make_layer(cfg: MoeConfig, seed: int = 0, layer: int = 0, bias: str | None =
         "experts": make_experts(cfg, seed, layer),
         "shared": make_shared(cfg, seed, layer),
     }
+
+
+def make_layer_device(cfg: MoeConfig, seed: int = 0, layer: int = 0, device="cuda", bias: str | None = None):
+    """A layer with the same distributions as make_layer, drawn on the GPU with torch's generator (fast enough
+    for the benchmark's 48-layer stack; the parity tests use make_layer, whose values the oracle regenerates).
+    Returns a dict of device tensors: router_w [E, H] fp32 ~ N(0, 0.02), router_b [E] fp32 (zero or the
+    Zipf(s) bias over a seeded rank permutation), experts [E, expert_bytes] uint8 and shared [expert_bytes]
+    uint8 in the canonical Q2 format (codes uniform in {0..3}, scales fp16(|N(0, 0.02)|))."""
+    import torch
+
+    E, H = cfg.n_experts, cfg.hidden
+    g = torch.Generator(device=device)
+    g.manual_seed(((seed * 1000003) ^ (layer * 7919) ^ 0x5EED) & 0x7FFFFFFFFFFF)
+    w = torch.randn((E, H), generator=g, device=device, dtype=torch.float32) * 0.02
+    kind = cfg.bias if bias is None else bias
+    if kind == "zero":
+        b = torch.zeros(E, dtype=torch.float32, device=device)
+    else:
+        beta = ZIPF_BETA if kind == "zipf" else ZIPF_BETA_COLD
+        ranks = torch.randperm(E, generator=g, device=device).to(torch.float64) + 1.0
+        b = (beta * (-ZIPF_S * torch.log(ranks))).to(torch.float32)
+    nblk = (3 * cfg.inter * H) // QBLOCK
+
+    def expert_blocks(n):
+        d = (torch.randn((n * nblk,), generator=g, device=device, dtype=torch.float32) * 0.02).abs().to(torch.float16)
+        qs = torch.randint(0, 256, (n * nblk, 8), generator=g, device=device, dtype=torch.uint8)
+        out = torch.empty((n * nblk, QBLOCK_BYTES), dtype=torch.uint8, device=device)
+        out[:, 0:2] = d.view(torch.uint8).view(n * nblk, 2)
+        out[:, 2:] = qs
+        return out.view(n, nblk * QBLOCK_BYTES)
+
+    experts = torch.cat([expert_blocks(min(64, E - e0)) for e0 in range(0, E, 64)])
+    shared = expert_blocks(1).view(-1)
+    return {"router_w": w, "router_b": b, "experts": experts, "shared": shared}

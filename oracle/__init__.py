@@ -66,6 +66,7 @@ def lib():
         L.orc_stack.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, ctypes.c_double, P, ctypes.c_double, P, P, P,
                                 ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         L.orc_num_threads.restype = i
+        L.orc_set_num_threads.argtypes = [i]
         _lib = L
     return _lib
 
@@ -80,6 +81,11 @@ def _c(a, dtype):
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the oracle's token loops (n < 1: all host threads)."""
+    lib().orc_set_num_threads(int(n))
 
 
 def half_to_double(bits: int) -> float:

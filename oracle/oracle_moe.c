@@ -358,3 +358,12 @@ int orc_num_threads(void) {
   return 1;
 #endif
 }
+
+/* Threads the oracle's token loops use from now on (n < 1: all host threads). */
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  omp_set_num_threads(n >= 1 ? n : omp_get_num_procs());
+#else
+  (void)n;
+#endif
+}

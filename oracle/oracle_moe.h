@@ -34,4 +34,5 @@ int orc_stack(int hidden, int inter, int n_experts, int top_k, int n_layers, int
               const uint8_t *const *shared, double eps, const int32_t *follow_idx, double tie_gap, double *resid,
               int32_t *idx_out, double *gap_out, int *n_followed, int *n_mismatch);
 int orc_num_threads(void);
+void orc_set_num_threads(int n);
 #endif
