@@ -5,11 +5,14 @@
 
 namespace moe {
 
+// The limits the header states: hidden and inter multiples of 128 (the packed layout's 128-wide block groups
+// along K) up to 4096; 1 <= top_k <= min(n_experts, 32) (one warp lane per selected expert); n_experts up to
+// 65535.
 static bool dims_ok(const moe_dims *d) {
   if (!d) return false;
   if (d->hidden < 128 || d->hidden > 4096 || d->hidden % 128) return false;
   if (d->inter < 128 || d->inter > 4096 || d->inter % 128) return false;
-  if (d->n_experts < 1 || d->n_experts > 4096) return false;
+  if (d->n_experts < 1 || d->n_experts > 65535) return false;
   if (d->top_k < 1 || d->top_k > d->n_experts || d->top_k > 32) return false;
   return true;
 }

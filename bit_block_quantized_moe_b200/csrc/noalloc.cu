@@ -94,7 +94,7 @@ bool noalloc_dims_ok(const moe_dims *d) {
   if (!d) return false;
   if (d->hidden < 128 || d->hidden > 4096 || d->hidden % 128) return false;
   if (d->inter < 128 || d->inter > 4096 || d->inter % 128) return false;
-  if (d->n_experts < 1 || d->n_experts > 4096) return false;
+  if (d->n_experts < 1 || d->n_experts > 65535) return false;
   if (d->top_k < 1 || d->top_k > d->n_experts || d->top_k > 32) return false;
   return true;
 }

@@ -44,8 +44,21 @@ struct CUstream_st;
 typedef struct CUstream_st *moe_stream_t;
 
 /* Layer dimensions.  The Q2 block is fixed at 32 weights.
- * Limits checked by every call: hidden and inter are multiples of 128 in
- * [128, 4096]; 1 <= n_experts <= 4096; 1 <= top_k <= min(n_experts, 32). */
+ * Limits checked by every call (MOE_ERR_ARG otherwise, sizes report 0):
+ *  - hidden and inter are multiples of 128 in [128, 4096].  The packed layout
+ *    groups four 32-weight blocks (128 weights) along the contraction
+ *    dimension: that group is one lane-fragment load, one TMA box and one
+ *    tensor-core K chunk, so a remainder of one to three blocks has no place
+ *    in it.  The pages' model (hidden 2048, expert intermediate 512 in this
+ *    library's synthetic stand-in) is far inside both bounds.
+ *  - 1 <= n_experts <= 65535 (the pages' model routes over 512 per layer).
+ *  - 1 <= top_k <= min(n_experts, 32): the selection keeps one warp lane per
+ *    selected expert (the pages' model selects 10).
+ * Which kernels run: T <= 8 with inter = 512, T * top_k <= 128 and
+ * n_experts <= 1024 takes one fused persistent kernel for the whole layer;
+ * other T <= 8 shapes take the routing kernels plus register-dequantising
+ * tensor-core expert kernels (slower, about 2x at the pages' shape); T > 8
+ * takes the tcgen05 prefill kernels. */
 typedef struct {
   int32_t hidden;    /* H: model width (router and expert input/output size) */
   int32_t inter;     /* I: expert intermediate size (gate/up rows, down columns) */
@@ -118,10 +131,13 @@ moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_ex
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t max_T);
 
 /* ---- routing ------------------------------------------------------------------
- * For each of T tokens: logits[e] = sum_h x[h] Wr[e][h] + bias[e] (fp32
- * accumulation); the top_k experts by logit, ties to the lower index, in
- * descending-logit order; weights = softmax over the selected logits (fp32),
- * which is the full softmax renormalised over the selected set.
+ * Every token goes to top_k of the n_experts routed experts (devlabs page,
+ * section 1, "MoE 专家分流": 10 of 512; Strata tuning page, section 2 model
+ * table).  The pages give no formula; this call computes, for each of T
+ * tokens: logits[e] = sum_h x[h] Wr[e][h] + bias[e] (fp32 accumulation); the
+ * top_k experts by logit, ties to the lower index, in descending-logit order;
+ * weights = softmax over the selected logits (fp32), which is the full softmax
+ * renormalised over the selected set.
  * x [T, hidden] bf16; topk_idx [T, top_k] int32 and topk_w [T, top_k] fp32 are
  * outputs.  T = 0 is a no-op. */
 moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_router *router, int32_t T,
@@ -160,6 +176,10 @@ moe_status moe_route_noalloc(const moe_dims *dims, const uint16_t *x, const moe_
                              int32_t *topk_idx, float *topk_w, moe_stream_t stream);
 
 /* ---- the layer ------------------------------------------------------------------
+ * The routed MoE FFN of the pages' model: top_k routed experts plus one shared
+ * expert per token (Strata tuning page, section 2 model table: 512 routed,
+ * top-10 + 1 shared), the experts computed straight from their 2-bit blocks
+ * (strata-mlx page, "它是什么", first bullet):
  * out[t] = shared(x[t]) + sum_j w[t,j] * expert_{idx[t,j]}(x[t]), with
  * expert(v) = Wd (silu(Wg v) * (Wu v)) and silu(z) = z / (1 + exp(-z)).
  * Rounding points: x is bf16; every dot product accumulates in fp32; the
@@ -173,7 +193,9 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
                              int32_t *topk_idx_out, float *topk_w_out, void *workspace, size_t ws_bytes,
                              moe_stream_t stream);
 
-/* The expert half of the layer for a routing decision made elsewhere:
+/* The expert half of the layer (the same model table: routed experts plus one
+ * shared expert, computed from their 2-bit blocks) for a routing decision made
+ * elsewhere:
  * dispatch (per-expert counts, offsets, stable token permutation), the routed
  * and shared SwiGLU experts and the weighted combine, with the rounding points
  * of moe_layer_forward.  topk_idx [T, top_k] int32 (each in [0, n_experts),

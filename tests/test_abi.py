@@ -42,7 +42,8 @@ def test_sizes(lib):
 
 @pytest.mark.parametrize("dims", [(2048, 512, 512, 0), (2048, 512, 512, 33), (2000, 512, 512, 10),
                                   (2048, 500, 512, 10), (8192, 512, 512, 10), (256, 128, 4, 5),
-                                  (256, 128, 5000, 10)])
+                                  (256, 128, 65536, 10), (96, 128, 16, 2), (4224, 128, 16, 2), (256, 4224, 16, 2),
+                                  (256, 160, 16, 2), (256, 128, 0, 1), (256, 128, 64, -1)])
 def test_bad_dims_rejected(lib, dims):
     d = B.moe_dims(*dims)
     assert B.moe_packed_expert_bytes(d) == 0
@@ -96,3 +97,14 @@ def test_workspace_size_never_shrinks_with_tokens(lib, dims):
         need = lib.moe_workspace_bytes(ctypes.byref(d), T)
         assert need >= prev, (dims, T, need, prev)
         prev = need
+
+
+@pytest.mark.parametrize("dims", [(128, 128, 1, 1), (4096, 4096, 16, 2), (256, 128, 65535, 32), (2048, 512, 512, 10),
+                                  (384, 640, 5000, 4)])
+def test_limits_accepted(lib, dims):
+    """The edges of the stated limits: multiples of 128 up to 4096, up to 65535 experts, up to 32 per token."""
+    d = B.moe_dims(*dims)
+    H, I = dims[0], dims[1]
+    assert B.moe_canonical_expert_bytes(d) == 3 * H * I // 32 * 10
+    assert B.moe_packed_expert_bytes(d) >= B.moe_canonical_expert_bytes(d)
+    assert B.moe_workspace_bytes(d, 8) > 0

@@ -60,6 +60,19 @@ def test_odd_shapes(dims):
         check_layer(cfg, w, x, y, idx, wts)
 
 
+def test_many_experts_beyond_the_fused_kernel():
+    """5000 routed experts (above the fused decode kernel's 1024): T = 3 takes the routing kernels plus the
+    register-dequant expert kernels, T = 13 and 300 the tcgen05 path; E near the 65535 limit only grows the
+    same per-expert work lists."""
+    cfg = MoeConfig("many experts", 128, 128, 5000, 4, 13, "zipf")
+    L, w = build_layer(cfg, seed=5)
+    for T in (3, 13, 300):
+        x = make_x(T, 128, seed=50 + T)
+        y, idx, wts = gpu_forward(L, x)
+        err, l2, flagged = check_layer(cfg, w, x, y, idx, wts)
+        print(f"E=5000 T={T}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
+
+
 def test_decode_window_full_size(full):
     L, w = full
     cfg = CONFIGS["decode"]
