@@ -709,11 +709,20 @@ def run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler):
     x = torch.from_numpy((make_x(T, H, seed=4000 + rank).astype(np.uint32) << 16).view(np.float32)).to(dev)
     resid = torch.empty_like(x)
     xn = torch.empty((T, H), dtype=torch.int16, device=dev)
+    xn2 = torch.empty_like(xn)
     y = torch.empty((T, H), dtype=torch.int16, device=dev)
     ws = torch.zeros(M.moe_workspace_bytes(dims, T), dtype=torch.uint8, device=dev)
     idx = torch.empty((T, cfg.top_k), dtype=torch.int32, device=dev)
 
-    def step(i):
+    def step(i):  # the residual and the next layer's RMSNorm in each layer's last kernel
+        resid.copy_(x)
+        M.moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6, stream=stream)
+        for l in range(L):
+            rw, rb, ex, sh = sets[l]
+            src, dst = (xn, xn2) if l % 2 == 0 else (xn2, xn)
+            M.moe_layer_forward_residual(dims, src, rw, rb, ex, sh, resid, dst, T, ws, 1e-6, stream=stream)
+
+    def step_unfused(i):  # the layer, then a separate residual + RMSNorm kernel
         resid.copy_(x)
         M.moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6, stream=stream)
         for l in range(L):
@@ -734,9 +743,10 @@ def run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler):
     torch.cuda.synchronize()
     K = max(1, min(args.steps, 5))
     win = sampler.window("stack 48 x T=1024") if sampler is not None else None
-    with torch.cuda.stream(stream):
-        secs = time_graph_steps(step, K, 3, stream, world, chunk=1, win=win)
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=1, win=win)
     ms = secs * 1e3 / K
+    secs_u = time_graph_steps(step_unfused, K, 3, stream, world, chunk=1)
+    ms_u = secs_u * 1e3 / K
     bytes_ = sum(layer_bytes(t, cfg.n_experts, H, T) for t in touched)
     flops = L * layer_flops(T, cfg.top_k, H, cfg.inter, cfg.n_experts)
     hbm = float(peaks["hbm_gbs"])
@@ -752,7 +762,10 @@ def run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler):
                     "RMSNorm eps 1e-6 + residual between layers, independent seeded weights per layer (24 GB)",
         "touched_experts_mean": float(np.mean(touched)), "bytes_per_step": bytes_, "flops_per_step": flops,
         "roofline_frac_of_measured": t_roof / (ms * 1e-3), "peak_source": peak_src,
-        "launches_per_layer": 12,
+        "step": "moe_layer_forward_residual per layer (residual + next RMSNorm in the combine)",
+        "launches_per_layer": 11,
+        "unfused": {"ms_per_step": ms_u, "ms_per_layer": ms_u / L, "launches_per_layer": 12,
+                    "step": "moe_layer_forward + moe_rmsnorm_residual per layer"},
     }
 
 

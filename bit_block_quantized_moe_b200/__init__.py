@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     moe_dispatch,
     moe_experts_forward,
     moe_layer_forward,
+    moe_layer_forward_residual,
     moe_pack_q2,
     moe_packed_expert_bytes,
     moe_rmsnorm_residual,

@@ -199,9 +199,18 @@ static moe_status check_layer_args(const moe_dims *dims, const uint16_t *x, cons
   return MOE_OK;
 }
 
+// Where the layer output goes: bf16 rows `out`, or (resid set) added in fp32 to the residual, whose RMSNorm
+// becomes the next layer's bf16 input x_norm.
+struct LayerOut {
+  uint16_t *out = nullptr;
+  float *resid = nullptr;
+  uint16_t *x_norm = nullptr;
+  float eps = 0.f;
+};
+
 // Dispatch, experts and combine for a routing already in ws.idx / ws.w.
 static cudaError_t run_experts(const moe_dims &d, const uint16_t *x, const moe_experts *experts,
-                               const moe_shared *shared, uint16_t *out, int T, Workspace &ws, cudaStream_t s,
+                               const moe_shared *shared, const LayerOut &lo, int T, Workspace &ws, cudaStream_t s,
                                bool bits_ready) {
   const PackedGeom G = packed_geom(d.hidden, d.inter);
   cudaError_t err = cudaSuccess;
@@ -213,7 +222,31 @@ static cudaError_t run_experts(const moe_dims &d, const uint16_t *x, const moe_e
     // few tokens: register-dequant tensor-core tiles of 8 tokens; otherwise the tcgen05 grouped GEMM
     err = T <= 8 ? launch_experts(d, G, ex, sh, x, T, ws, s) : launch_tc_experts(d, G, ex, sh, x, T, ws, s);
   }
-  if (err == cudaSuccess) err = launch_combine(d, T, ws, out, s);
+  if (err == cudaSuccess)
+    err = lo.resid ? launch_combine_rmsnorm(d, T, ws, lo.resid, lo.x_norm, lo.eps, s) : launch_combine(d, T, ws, lo.out, s);
+  return err;
+}
+
+// The layer for x (routing, experts, combine) into `lo`.
+static cudaError_t run_layer(const moe_dims &d, const uint16_t *x, const moe_router *router,
+                             const moe_experts *experts, const moe_shared *shared, const LayerOut &lo, int T,
+                             int32_t *topk_idx_out, float *topk_w_out, Workspace &ws, cudaStream_t s) {
+  if (topk_idx_out) ws.idx = topk_idx_out;
+  if (topk_w_out) ws.w = topk_w_out;
+  if (decode_fused_supported(d, T)) {
+    // The fused kernel writes the routing copies as a pair (both pointers or neither): when only one is
+    // requested, the other goes to the workspace's own [T, top_k] buffer.
+    const bool copies = topk_idx_out || topk_w_out;
+    // with a residual the fused kernel leaves the fp32 layer output in the workspace's expert-output rows
+    cudaError_t err = launch_decode_fused(d, x, router->w, router->bias, static_cast<const uint8_t *>(experts->packed),
+                                          static_cast<const uint8_t *>(shared->packed), T, ws,
+                                          copies ? ws.idx : nullptr, copies ? ws.w : nullptr,
+                                          lo.resid ? nullptr : lo.out, lo.resid ? ws.y : nullptr, s);
+    if (err == cudaSuccess && lo.resid) err = launch_rmsnorm_residual_f32(lo.resid, ws.y, lo.x_norm, T, d.hidden, lo.eps, s);
+    return err;
+  }
+  cudaError_t err = launch_route(d, x, router->w, router->bias, T, ws, true, s);
+  if (err == cudaSuccess) err = run_experts(d, x, experts, shared, lo, T, ws, s, true);
   return err;
 }
 
@@ -231,20 +264,37 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Workspace ws;
   workspace_layout(*dims, T, workspace, &ws);
-  if (topk_idx_out) ws.idx = topk_idx_out;
-  if (topk_w_out) ws.w = topk_w_out;
-  if (decode_fused_supported(*dims, T)) {
-    // The fused kernel writes the routing copies as a pair (both pointers or neither): when only one is
-    // requested, the other goes to the workspace's own [T, top_k] buffer.
-    const bool copies = topk_idx_out || topk_w_out;
-    return cuda_status(launch_decode_fused(*dims, x, router->w, router->bias,
-                                           static_cast<const uint8_t *>(experts->packed),
-                                           static_cast<const uint8_t *>(shared->packed), T, ws,
-                                           copies ? ws.idx : nullptr, copies ? ws.w : nullptr, out, s));
-  }
-  cudaError_t err = launch_route(*dims, x, router->w, router->bias, T, ws, true, s);
-  if (err == cudaSuccess) err = run_experts(*dims, x, experts, shared, out, T, ws, s, true);
-  return cuda_status(err);
+  LayerOut lo;
+  lo.out = out;
+  return cuda_status(run_layer(*dims, x, router, experts, shared, lo, T, topk_idx_out, topk_w_out, ws, s));
+}
+
+static bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + nb && y < x + na;
+}
+
+moe_status moe_layer_forward_residual(const moe_dims *dims, const uint16_t *x_norm_in, const moe_router *router,
+                                      const moe_experts *experts, const moe_shared *shared, float *resid,
+                                      uint16_t *x_norm_out, float eps, int32_t T, int32_t *topk_idx_out,
+                                      float *topk_w_out, void *workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (!router || !(eps >= 0.f)) return MOE_ERR_ARG;
+  moe_status st = check_layer_args(dims, x_norm_in, experts, shared, x_norm_out, T, workspace, ws_bytes);
+  if (st != MOE_OK || T == 0) return st;
+  if (!router->w || !resid) return MOE_ERR_ARG;
+  if (!aligned16(router->w) || !aligned16(resid)) return MOE_ERR_ALIGN;
+  const size_t xb = (size_t)T * dims->hidden * 2, rb = (size_t)T * dims->hidden * 4;
+  if (overlaps(resid, rb, x_norm_in, xb) || overlaps(resid, rb, x_norm_out, xb)) return MOE_ERR_ARG;
+  const moe_status dev = device_ok();
+  if (dev != MOE_OK) return dev;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Workspace ws;
+  workspace_layout(*dims, T, workspace, &ws);
+  LayerOut lo;
+  lo.resid = resid;
+  lo.x_norm = x_norm_out;
+  lo.eps = eps;
+  return cuda_status(run_layer(*dims, x_norm_in, router, experts, shared, lo, T, topk_idx_out, topk_w_out, ws, s));
 }
 
 moe_status moe_experts_forward(const moe_dims *dims, const uint16_t *x, const int32_t *topk_idx,
@@ -260,7 +310,9 @@ moe_status moe_experts_forward(const moe_dims *dims, const uint16_t *x, const in
   workspace_layout(*dims, T, workspace, &ws);
   ws.idx = const_cast<int32_t *>(topk_idx);
   ws.w = const_cast<float *>(topk_w);
-  return cuda_status(run_experts(*dims, x, experts, shared, out, T, ws, s, false));
+  LayerOut lo;
+  lo.out = out;
+  return cuda_status(run_experts(*dims, x, experts, shared, lo, T, ws, s, false));
 }
 
 moe_status moe_dispatch(const moe_dims *dims, const int32_t *topk_idx, int32_t T, int32_t *counts,

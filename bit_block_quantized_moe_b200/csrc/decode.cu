@@ -68,7 +68,8 @@ struct DecodeArgs {
   uint64_t *gbar;      // monotonic grid-barrier arrival counter
   int32_t *idx_out;    // optional [T][k]
   float *w_out;        // optional [T][k]
-  uint16_t *out;       // [T][H]
+  uint16_t *out;       // [T][H] bf16, or
+  float *out_f32;      // [T][H] fp32 (when set: the layer output is not rounded)
   uint32_t *status;
   int ns;              // ring stages: nw warps x (ns / nw) private slots each
   int nw;              // warps that stream and compute expert stages
@@ -507,8 +508,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     for (int hf = 0; hf < 2; ++hf) {
       const int n = 2 * c + hf;
       if (n < T) {
-        a.out[(size_t)n * H + r0] = float_to_bf16_bits(o[hf]);
-        a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 + hf]);
+        if (a.out_f32) {
+          a.out_f32[(size_t)n * H + r0] = o[hf];
+          a.out_f32[(size_t)n * H + r0 + 8] = o[2 + hf];
+        } else {
+          a.out[(size_t)n * H + r0] = float_to_bf16_bits(o[hf]);
+          a.out[(size_t)n * H + r0 + 8] = float_to_bf16_bits(o[2 + hf]);
+        }
       }
     }
   };
@@ -585,7 +591,7 @@ size_t decode_counter_words(const moe_dims &d) { return (size_t)d.hidden / 16 + 
 
 cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias,
                                 const uint8_t *experts, const uint8_t *shared, int T, const Workspace &ws,
-                                int32_t *idx_out, float *w_out, uint16_t *out, cudaStream_t s) {
+                                int32_t *idx_out, float *w_out, uint16_t *out, float *out_f32, cudaStream_t s) {
   const PackedGeom G = packed_geom(d.hidden, d.inter);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -633,6 +639,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   a.idx_out = idx_out;
   a.w_out = w_out;
   a.out = out;
+  a.out_f32 = out_f32;
   a.status = ws.status;
   a.ns = ns;
   a.nw = nw;

@@ -62,7 +62,7 @@ size_t decode_partial_floats(const moe_dims &d, int T);
 size_t decode_counter_words(const moe_dims &d);
 cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias,
                                 const uint8_t *experts, const uint8_t *shared, int T, const Workspace &ws,
-                                int32_t *idx_out, float *w_out, uint16_t *out, cudaStream_t s);
+                                int32_t *idx_out, float *w_out, uint16_t *out, float *out_f32, cudaStream_t s);
 bool router_tc_supported(const moe_dims &d, int T);
 int router_tc_ksplit(const moe_dims &d, int T);
 size_t router_tc_partial_bytes_max();
@@ -70,5 +70,9 @@ cudaError_t launch_router_tc(const moe_dims &d, const uint16_t *x, const float *
                              const Workspace &ws, cudaStream_t s);
 cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,
                                     cudaStream_t s);
+cudaError_t launch_rmsnorm_residual_f32(float *resid, const float *y, uint16_t *x_norm, int T, int H, float eps,
+                                        cudaStream_t s);
+cudaError_t launch_combine_rmsnorm(const moe_dims &d, int T, const Workspace &ws, float *resid, uint16_t *x_norm,
+                                   float eps, cudaStream_t s);
 
 }  // namespace moe

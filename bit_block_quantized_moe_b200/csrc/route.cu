@@ -534,9 +534,27 @@ cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16
 }
 
 // ---------------------------------------------------------------------------
-// Between layers: resid += y (optional); x_norm = bf16(resid * rsqrt(mean(resid^2) + eps)).
-__global__ void __launch_bounds__(256) rmsnorm_residual_kernel(float *__restrict__ resid,
-                                                               const uint16_t *__restrict__ y,
+// Between layers: resid += y (optional); x_norm = bf16(resid * rsqrt(mean(resid^2) + eps)).  One CTA of 256
+// threads per token; the sum of squares is reduced in a fixed order (deterministic).
+
+// Sum over the CTA (blockDim.x a multiple of 32, at most 1024); every thread gets the total.
+__device__ __forceinline__ float block_sum(float v, float *part) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float u = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
+    if (threadIdx.x == 0) part[32] = u;
+  }
+  __syncthreads();
+  return part[32];
+}
+
+template <typename YT>  // layer output type: uint16_t (bf16 bits) or float
+__global__ void __launch_bounds__(256) rmsnorm_residual_kernel(float *__restrict__ resid, const YT *__restrict__ y,
                                                                uint16_t *__restrict__ x_norm, int H, float eps) {
   const int t = blockIdx.x;
   float *r = resid + (size_t)t * H;
@@ -544,30 +562,87 @@ __global__ void __launch_bounds__(256) rmsnorm_residual_kernel(float *__restrict
   for (int i = threadIdx.x; i < H; i += blockDim.x) {
     float v = r[i];
     if (y) {
-      v += bf16_bits_to_float(y[(size_t)t * H + i]);
+      const YT yv = y[(size_t)t * H + i];
+      if constexpr (sizeof(YT) == 2) v += bf16_bits_to_float(yv);
+      else v += yv;
       r[i] = v;
     }
     ss = fmaf(v, v, ss);
   }
-  __shared__ float part[32];
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if (threadIdx.x == 0) part[0] = v;
-  }
-  __syncthreads();
-  const float scale = 1.0f / sqrtf(part[0] / (float)H + eps);
+  __shared__ float part[33];
+  const float scale = 1.0f / sqrtf(block_sum(ss, part) / (float)H + eps);
   for (int i = threadIdx.x; i < H; i += blockDim.x) x_norm[(size_t)t * H + i] = float_to_bf16_bits(r[i] * scale);
 }
 
 cudaError_t launch_rmsnorm_residual(float *resid, const uint16_t *y, uint16_t *x_norm, int T, int H, float eps,
                                     cudaStream_t s) {
-  rmsnorm_residual_kernel<<<T, 256, 0, s>>>(resid, y, x_norm, H, eps);
+  rmsnorm_residual_kernel<uint16_t><<<T, 256, 0, s>>>(resid, y, x_norm, H, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm_residual_f32(float *resid, const float *y, uint16_t *x_norm, int T, int H, float eps,
+                                        cudaStream_t s) {
+  rmsnorm_residual_kernel<float><<<T, 256, 0, s>>>(resid, y, x_norm, H, eps);
+  return cudaGetLastError();
+}
+
+// Combine fused with the residual and the next layer's RMSNorm (one CTA per token): y = Y_shared[t] +
+// sum_j w[t,j] Y[slot(t,j)] in the combine's fixed order (fp32, never rounded), resid += y, x_norm =
+// bf16(resid / sqrt(mean(resid^2) + eps)).
+__global__ void __launch_bounds__(256) combine_rmsnorm_kernel(const float *__restrict__ Y,
+                                                              const int32_t *__restrict__ slot_pos,
+                                                              const float *__restrict__ topk_w, int T, int k, int H,
+                                                              float *__restrict__ resid, uint16_t *__restrict__ x_norm,
+                                                              float eps) {
+  const int t = blockIdx.x;
+  float4 *r4 = reinterpret_cast<float4 *>(resid + (size_t)t * H);
+  __shared__ int pos_s[32];
+  __shared__ float w_s[32];
+  __shared__ float part[33];
+  if (threadIdx.x < k) {
+    pos_s[threadIdx.x] = slot_pos[(size_t)t * k + threadIdx.x];
+    w_s[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int c4 = threadIdx.x; c4 < H / 4; c4 += blockDim.x) {
+    float4 acc = reinterpret_cast<const float4 *>(Y + ((size_t)T * k + t) * H)[c4];
+    for (int j = 0; j < k; ++j) {
+      const int pos = pos_s[j];
+      if (pos < 0) continue;  // an invalid slot adds nothing
+      const float wj = w_s[j];
+      const float4 v = reinterpret_cast<const float4 *>(Y + (size_t)pos * H)[c4];
+      acc.x = fmaf(wj, v.x, acc.x);
+      acc.y = fmaf(wj, v.y, acc.y);
+      acc.z = fmaf(wj, v.z, acc.z);
+      acc.w = fmaf(wj, v.w, acc.w);
+    }
+    float4 rv = r4[c4];
+    rv.x += acc.x;
+    rv.y += acc.y;
+    rv.z += acc.z;
+    rv.w += acc.w;
+    r4[c4] = rv;
+    ss = fmaf(rv.x, rv.x, ss);
+    ss = fmaf(rv.y, rv.y, ss);
+    ss = fmaf(rv.z, rv.z, ss);
+    ss = fmaf(rv.w, rv.w, ss);
+  }
+  const float scale = 1.0f / sqrtf(block_sum(ss, part) / (float)H + eps);
+  for (int c4 = threadIdx.x; c4 < H / 4; c4 += blockDim.x) {
+    const float4 rv = r4[c4];
+    uint2 o;
+    o.x = pack_bf16x2(rv.x * scale, rv.y * scale);
+    o.y = pack_bf16x2(rv.z * scale, rv.w * scale);
+    reinterpret_cast<uint2 *>(x_norm + (size_t)t * H)[c4] = o;
+  }
+}
+
+cudaError_t launch_combine_rmsnorm(const moe_dims &d, int T, const Workspace &ws, float *resid, uint16_t *x_norm,
+                                   float eps, cudaStream_t s) {
+  trace_mark(MOE_KERNEL_COMBINE, false, s);
+  combine_rmsnorm_kernel<<<T, 256, 0, s>>>(ws.y, ws.slot_pos, ws.w, T, d.top_k, d.hidden, resid, x_norm, eps);
+  trace_mark(MOE_KERNEL_COMBINE, true, s);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,14 @@ class Q2MoeLayer:
                             self.workspace, topk_idx, topk_w, stream)
         return out
 
+    def forward_residual(self, x_norm, resid, x_norm_out, eps=1e-6, topk_idx=None, topk_w=None, stream=None):
+        """One stacked layer: resid += layer(x_norm); x_norm_out = bf16(RMSNorm(resid))."""
+        T = x_norm.shape[0]
+        self.reserve(T)
+        B.moe_layer_forward_residual(self.dims, x_norm, self.router_w, self.router_b, self.experts, self.shared, resid,
+                                     x_norm_out, T, self.workspace, eps, topk_idx, topk_w, stream)
+        return x_norm_out
+
     def experts_forward(self, x, topk_idx, topk_w, out=None, stream=None):
         T = x.shape[0]
         self.reserve(T)

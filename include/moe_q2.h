@@ -193,6 +193,26 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
                              int32_t *topk_idx_out, float *topk_w_out, void *workspace, size_t ws_bytes,
                              moe_stream_t stream);
 
+/* One layer of a stack of layers (the pages' model stacks 48 of them, Strata
+ * tuning page, section 2 model table), with the residual stream and the next
+ * layer's normalisation done by the layer's own last kernel:
+ *   y = the layer of moe_layer_forward applied to x_norm_in;
+ *   resid += y                    (fp32; y is not rounded to bf16 on the way)
+ *   x_norm_out = bf16(resid / sqrt(mean(resid^2) + eps))   (unit gain, nearest even)
+ * resid [T, hidden] fp32 (in/out); x_norm_in / x_norm_out [T, hidden] bf16,
+ * which must not overlap each other or resid.  A stack is
+ *   moe_rmsnorm_residual(resid = x, NULL, x_norm);  then per layer
+ *   moe_layer_forward_residual(layer, x_norm, resid, x_norm') with x_norm and
+ *   x_norm' swapped between layers.
+ * It equals moe_layer_forward followed by moe_rmsnorm_residual except that
+ * the layer output reaches the residual unrounded, one launch fewer per
+ * layer for T > 8 and one bf16 [T, hidden] round trip less.  eps >= 0.
+ * Other arguments and errors as moe_layer_forward. */
+moe_status moe_layer_forward_residual(const moe_dims *dims, const uint16_t *x_norm_in, const moe_router *router,
+                                      const moe_experts *experts, const moe_shared *shared, float *resid,
+                                      uint16_t *x_norm_out, float eps, int32_t T, int32_t *topk_idx_out,
+                                      float *topk_w_out, void *workspace, size_t ws_bytes, moe_stream_t stream);
+
 /* The expert half of the layer (the same model table: routed experts plus one
  * shared expert, computed from their 2-bit blocks) for a routing decision made
  * elsewhere:

@@ -242,30 +242,30 @@ def test_routing_copies_one_at_a_time(full):
     assert torch.equal(y1, y2)
 
 
-def test_stack_48_layers_against_oracle_stack():
-    """The 48-layer stack (the pages' model depth) at T = 1024, end to end: x_0 = x; layer l reads
-    bf16(RMSNorm(r_l)); r_{l+1} = r_l + y_l, the residual fp32 on the GPU and fp64 in the oracle.  The GPU runs all
-    1024 tokens through all 48 layers with no re-anchoring; the oracle stack carries 256 sampled tokens through
-    the same 48 layers from the same x.
+def _stack_against_oracle(L, fused):
+    """A stack of L full-size layers at T = 1024, end to end: x_0 = x; layer l reads bf16(RMSNorm(r_l));
+    r_{l+1} = r_l + y_l, the residual fp32 on the GPU and fp64 in the oracle.  The GPU runs all 1024 tokens
+    through all L layers with no re-anchoring (fused: moe_layer_forward_residual; else moe_layer_forward +
+    moe_rmsnorm_residual); the oracle stack carries 256 sampled tokens through the same layers from the same x.
 
-    Every routing decision the GPU takes in the stack is checked against the oracle's routing of the GPU's own
-    layer input (sets bit-exact except near-ties).  The two trajectories' layer inputs drift apart by the
-    accumulated rounding of earlier layers, so a token whose margin is below that drift may take a different set
-    on the two sides; there the oracle stack takes the GPU's set (counted and printed).  The final residuals
-    must agree within max|dr| / max|r| <= 1e-2; the drift of the bf16 layer input is printed every 8 layers."""
+    Every routing decision the GPU takes is checked against the oracle's routing of the GPU's own layer input
+    (sets bit-exact except near-ties).  The two trajectories' layer inputs drift apart by the accumulated
+    rounding of earlier layers, so a token whose margin is below that drift may take a different set on the two
+    sides; there the oracle stack takes the GPU's set (counted and printed).  The final residuals must agree
+    within max|dr| / max|r| <= 1e-2; the drift of the bf16 layer input is printed every 8 layers."""
     import math
 
     from bit_block_quantized_moe_b200 import moe_rmsnorm_residual
     from gen import make_layer
 
     cfg = CONFIGS["stack"]
-    T, H, L, k = cfg.tokens, cfg.hidden, cfg.layers, cfg.top_k
-    assert L == 48
+    T, H, k = cfg.tokens, cfg.hidden, cfg.top_k
     rng = np.random.default_rng(3)
     sample = np.sort(rng.choice(T, 256, replace=False))
     x0 = make_x(cfg, seed=0)
     resid = torch.from_numpy(bf16_to_f32(x0)).cuda()
     xn = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    xn2 = torch.empty_like(xn)
     moe_rmsnorm_residual(resid, None, xn, T, H, 1e-6)
     idx_g = np.empty((L, sample.size, k), dtype=np.int32)
     w_g = np.empty((L, sample.size, k), dtype=np.float32)
@@ -274,20 +274,24 @@ def test_stack_48_layers_against_oracle_stack():
         Lyr, _ = build_layer(cfg, layer=layer)
         idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
         wts = torch.zeros((T, k), dtype=torch.float32, device="cuda")
-        y = Lyr.forward(xn, topk_idx=idx, topk_w=wts)
+        xn_g[layer] = xn.cpu().numpy().view(np.uint16)[sample]
+        if fused:
+            Lyr.forward_residual(xn, resid, xn2, 1e-6, topk_idx=idx, topk_w=wts)
+            xn, xn2 = xn2, xn
+        else:
+            y = Lyr.forward(xn, topk_idx=idx, topk_w=wts)
+            moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6)  # r += y; the next layer's input
         torch.cuda.synchronize()
         Lyr.check_status()
-        xn_g[layer] = xn.cpu().numpy().view(np.uint16)[sample]
         idx_g[layer] = idx.cpu().numpy()[sample]
         w_g[layer] = wts.cpu().numpy()[sample]
-        moe_rmsnorm_residual(resid, y, xn, T, H, 1e-6)  # r += y; the next layer's input
         del Lyr
     torch.cuda.synchronize()
     r_gpu = resid.cpu().numpy()[sample].astype(np.float64)
 
     r = None
     followed, flagged = 0, 0
-    bounds = [0, 8, 16, 24, 32, 40, 47, 48]
+    bounds = sorted(set(list(range(0, L, 8)) + [max(L - 1, 0), L]))
     for c0, c1 in zip(bounds[:-1], bounds[1:]):
         lays = [make_layer(cfg, seed=0, layer=l) for l in range(c0, c1)]
         # the layer input of layer c0 on both sides
@@ -304,10 +308,55 @@ def test_stack_48_layers_against_oracle_stack():
         del lays
     err = np.max(np.abs(r_gpu - r)) / np.max(np.abs(r))
     rel_l2 = np.linalg.norm(r_gpu - r) / np.linalg.norm(r)
-    print(f"stack of 48 layers, 256 tokens: final residual max|dr|/max|r| = {err:.3e}, relL2 {rel_l2:.3e}; "
-          f"near-tie routing differences on the GPU's own inputs: {flagged}; (layer, token) pairs where the two "
-          f"trajectories routed differently and the oracle took the GPU's set: {followed} of {L * sample.size}")
+    print(f"stack of {L} layers ({'fused residual' if fused else 'layer + rmsnorm_residual'}), 256 tokens: final "
+          f"residual max|dr|/max|r| = {err:.3e}, relL2 {rel_l2:.3e}; near-tie routing differences on the GPU's own "
+          f"inputs: {flagged}; (layer, token) pairs where the two trajectories routed differently and the oracle "
+          f"took the GPU's set: {followed} of {L * sample.size}")
     assert err <= 1e-2
+
+
+def test_stack_48_layers_against_oracle_stack():
+    """The pages' model depth: 48 layers (Strata tuning page, section 2 model table), through the fused
+    residual call the stack benchmark times."""
+    _stack_against_oracle(48, fused=True)
+
+
+def test_stack_6_layers_layer_plus_rmsnorm_against_oracle_stack():
+    _stack_against_oracle(6, fused=False)
+
+
+@pytest.mark.parametrize("T", [3, 5, 100, 1024])
+def test_layer_forward_residual(full, T):
+    """resid += layer(x_norm) and the next RMSNorm in the layer's last kernel: against moe_layer_forward +
+    moe_rmsnorm_residual (which rounds y to bf16 first) and against the oracle's layer output."""
+    from bit_block_quantized_moe_b200 import moe_rmsnorm_residual
+
+    L, w = full
+    cfg = CONFIGS["prefill"]
+    H = cfg.hidden
+    rng = np.random.default_rng(T)
+    r0 = torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)).cuda()
+    xn = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    moe_rmsnorm_residual(r0.clone(), None, xn, T, H, 1e-6)
+    ra, xa = r0.clone(), torch.empty_like(xn)
+    idx = torch.full((T, cfg.top_k), -1, dtype=torch.int32, device="cuda")
+    wts = torch.zeros((T, cfg.top_k), dtype=torch.float32, device="cuda")
+    L.forward_residual(xn, ra, xa, 1e-6, topk_idx=idx, topk_w=wts)
+    y = L.forward(xn)
+    rb, xb = r0.clone(), torch.empty_like(xn)
+    moe_rmsnorm_residual(rb, y, xb, T, H, 1e-6)
+    torch.cuda.synchronize()
+    L.check_status()
+    ya = (ra - r0).cpu().numpy().astype(np.float64)
+    ymax = float(np.max(np.abs(ya)))
+    # the unfused pair differs only by y's bf16 rounding
+    assert torch.max(torch.abs(ra - rb)).item() <= 2.0 ** -8 * ymax + 1e-6
+    xn_np = xn.cpu().numpy().view(np.uint16)
+    err, l2, flagged = check_layer(cfg, w, xn_np, ya, idx.cpu().numpy(), wts.cpu().numpy())
+    want = oracle.rmsnorm(ra.cpu().numpy().astype(np.float64), 1e-6)
+    got = bf16_to_f32(xa.cpu().numpy().view(np.uint16))
+    assert np.max(np.abs(got - want) / np.maximum(np.abs(want), 1e-3)) < 2 ** -8
+    print(f"fused residual T={T}: layer max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}")
 
 
 def test_prefill_chunk_32768(full):
