@@ -484,12 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     float o[4] = {0.f, 0.f, 0.f, 0.f};
     const float *pp = a.partial + (size_t)tile * 128 + lane * 4;
     int e2 = 0;
-    for (; e2 + 4 <= nent; e2 += 4) {  // four loads in flight, summed in expert order
-      float4 v[4];
+    for (; e2 < nent; e2 += 16) {  // up to sixteen loads in flight, summed in expert order
+      float4 v[16];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = ldg_cg_f4(pp + (size_t)(e2 + u) * G.dn_units * 128);
+      for (int u = 0; u < 16; ++u)
+        v[u] = e2 + u < nent ? ldg_cg_f4(pp + (size_t)(e2 + u) * G.dn_units * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 16; ++u) {
         o[0] += v[u].x;
         o[1] += v[u].y;
         o[2] += v[u].z;

@@ -22,7 +22,10 @@
 //                     from shared memory), fp32 accumulators in tensor
 //                     memory, one commit per chunk.  It waits only on the A
 //                     stage: the dequant warps passed the chunk's TMA barrier
-//                     before filling it, which orders the B rows too;
+//                     before filling it, which orders the B rows too.  The
+//                     whole warp runs the loop on warp-uniform values and one
+//                     elected lane issues (a lane-0-only loop issues the same
+//                     MMAs about 20% slower; the producer warp likewise);
 //   4 epilogue warps: tcgen05.ld the accumulators; gate/up writes
 //                     h = silu(g) * u (bf16, each lane one SiLU per pair of
 //                     token columns), down writes the fp32 expert output rows
@@ -160,18 +163,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
   const uint32_t tbase = B.tmem;
 
   if (warp == kWarpProducer) {
-    if (lane == 0) {
-      int cnt = 0;
-      for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
-        const int4 it = a.items[w / a.mgroups];
-        const int mt0 = (w % a.mgroups) * kMT;
-        const int bsel = it.z <= 16 ? 0 : (it.z <= 32 ? 1 : (it.z <= 64 ? 2 : 3));
-        const int nrows = 16 << bsel;
-        const CUtensorMap *amap = it.x == a.E ? &maps.a_shared : &maps.a_routed;
-        const int ae = it.x == a.E ? 0 : it.x;
-        for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
-          const int s = cnt % kStages;
-          if (!waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) continue;
+    // The whole warp runs the loop; one elected lane issues the copies.
+    int cnt = 0;
+    for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+      const int4 it = a.items[w / a.mgroups];
+      const int mt0 = (w % a.mgroups) * kMT;
+      const int bsel = it.z <= 16 ? 0 : (it.z <= 32 ? 1 : (it.z <= 64 ? 2 : 3));
+      const int nrows = 16 << bsel;
+      const CUtensorMap *amap = it.x == a.E ? &maps.a_shared : &maps.a_routed;
+      const int ae = it.x == a.E ? 0 : it.x;
+      for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
+        const int s = cnt % kStages;
+        if (!waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) continue;
+        if (elect_one()) {
           uint8_t *st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&B.full[s], (uint32_t)(kABytes + 2 * nrows * 128));
           // kMT x 8 units; units past the expert's last tile read as zeros (tensor-map bounds)
@@ -179,30 +183,29 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
           for (int sub = 0; sub < 2; ++sub)
             tma_load_2d(st + kABytes + sub * kBSub, &maps.b[bsel], kc * 128 + sub * 64, it.y, &B.full[s]);
         }
+        __syncwarp();
       }
-      // every copy issued must land before the CTA exits
-      for (int c2 = max(0, cnt - kStages); c2 < cnt; ++c2) waitb(&B.full[c2 % kStages], (c2 / kStages) & 1, B, a.status);
     }
+    // every copy issued must land before the CTA exits
+    for (int c2 = max(0, cnt - kStages); c2 < cnt; ++c2) waitb(&B.full[c2 % kStages], (c2 / kStages) & 1, B, a.status);
   } else if (warp == kWarpMMA) {
-    if (lane == 0) {
-      int cnt = 0, dcnt = 0;
-      for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
-        const int4 it = a.items[w / a.mgroups];
-        const int N = max(16, (it.z + 15) & ~15);
-        const uint32_t idesc = umma_idesc_bf16(128, N);
-        const int db = dcnt & 1;
-        waitb(&B.dempty[db], ((dcnt >> 1) & 1) ^ 1, B, a.status);
+    // The whole warp runs the loop on warp-uniform values; one elected lane issues the MMAs and commits.
+    int cnt = 0, dcnt = 0;
+    for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+      const int4 it = a.items[w / a.mgroups];
+      const int N = max(16, (it.z + 15) & ~15);
+      const uint32_t idesc = umma_idesc_bf16(128, N);
+      const int db = dcnt & 1;
+      waitb(&B.dempty[db], ((dcnt >> 1) & 1) ^ 1, B, a.status);
+      tc_fence_after();
+      const uint32_t dcol = tbase + db * kDCols;
+      for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
+        const int s = cnt % kStages, sa = cnt % kAStages;
+        waitb(&B.afull[sa], (cnt / kAStages) & 1, B, a.status);
         tc_fence_after();
-        const uint32_t dcol = tbase + db * kDCols;
-        for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
-          const int s = cnt % kStages, sa = cnt % kAStages;
-          // Every dequant warp waited on this chunk's TMA barrier before its arrival here, so the
-          // B rows of stage s are in shared memory as well.
-          waitb(&B.afull[sa], (cnt / kAStages) & 1, B, a.status);
-          tc_fence_after();
-          // K step j: 64-column half j / 4 of the stage's B rows, 32 bytes per step inside the half
-          const uint64_t bdesc0 = umma_sdesc_sw128(smem_u32(smem + s * kStageBytes + kABytes));
-          const uint32_t acol = tbase + kTmemA0 + sa * kMT * 64;
+        const uint64_t bdesc0 = umma_sdesc_sw128(smem_u32(smem + s * kStageBytes + kABytes));
+        const uint32_t acol = tbase + kTmemA0 + sa * kMT * 64;
+        if (elect_one()) {
 #pragma unroll
           for (int m = 0; m < kMT; ++m)
 #pragma unroll
@@ -211,13 +214,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
                       bdesc0 + (uint64_t)((j >> 2) * (kBSub >> 4) + (j & 3) * 2), idesc, (kc | j) != 0);
           umma_commit(&B.aempty[sa]);
         }
-        umma_commit(&B.dfull[db]);
-        ++dcnt;
+        __syncwarp();
       }
-      // all MMAs issued by this thread have completed before tensor memory is released
+      if (elect_one()) umma_commit(&B.dfull[db]);
+      __syncwarp();
+      ++dcnt;
+    }
+    // all MMAs issued by this warp have completed before tensor memory is released
+    if (elect_one()) {
       umma_commit(&B.done);
       if (!mbar_wait(&B.done, 0)) set_status(a.status, kStatusTimeout);
     }
+    __syncwarp();
   } else if (warp < kWarpEpi0) {
     // ---- dequant warps: 4 per TMEM lane quadrant (the quadrant holds units 2q, 2q + 1 of each M tile):
     // with two M tiles one whole unit each, with one tile half a unit (2 of its 4 blocks) each ----
