@@ -545,15 +545,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
       *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
       // Count the contribution; the warp that brings the tile's last one sums all its
-      // partials in expert order right away and writes the output rows.
+      // partials in expert order right away and writes the output rows.  The warp sync orders
+      // every lane's partial store before lane 0's release; the count is one acquire-release
+      // atomic at GPU scope, so the last contributor also acquires every other partial (a full
+      // fence on both sides cost 0.3-0.5 us more per step).
       __syncwarp();
       int last = 0;
-      if (lane == 0) {
-        __threadfence();
-        last = atomicAdd(&a.tile_cnt[tile], 1u) == (uint32_t)(nent - 1);
-      }
+      if (lane == 0) last = atom_add_acq_rel_gpu(&a.tile_cnt[tile], 1u) == (uint32_t)(nent - 1);
       if (__shfl_sync(0xffffffffu, last, 0)) {
-        __threadfence();
+        __syncwarp();
         reduce_tile(tile);
       }
     }
