@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     moe_rmsnorm_residual,
     moe_route,
     moe_route_noalloc,
+    moe_set_cold_expert_tokens,
     moe_status_str,
     moe_trace_kernel,
     MOE_KERNEL,

@@ -49,6 +49,7 @@ EXPORTED = [
     "moe_dispatch",
     "moe_rmsnorm_residual",
     "moe_trace_kernel",
+    "moe_set_cold_expert_tokens",
     "moe_check_status",
     "moe_status_str",
 ]
@@ -91,6 +92,8 @@ def lib():
         L.moe_rmsnorm_residual.argtypes = [P, P, P, i32, i32, ctypes.c_float, P]
         L.moe_trace_kernel.restype = ctypes.c_int
         L.moe_trace_kernel.argtypes = [i32, P, P]
+        L.moe_set_cold_expert_tokens.restype = ctypes.c_int
+        L.moe_set_cold_expert_tokens.argtypes = [i32]
         L.moe_check_status.restype = ctypes.c_int
         L.moe_check_status.argtypes = [P, P]
         L.moe_status_str.restype = ctypes.c_char_p
@@ -223,6 +226,12 @@ def moe_trace_kernel(kernel_id: int, before=None, after=None):
     b = None if before is None else before.cuda_event
     a = None if after is None else after.cuda_event
     _check(lib().moe_trace_kernel(int(kernel_id), b, a), "moe_trace_kernel")
+
+
+def moe_set_cold_expert_tokens(max_tokens: int):
+    """Per host thread: in a prefill chunk, experts with at most max_tokens tokens run on the register-dequant
+    kernels (0, the default: every expert on the tcgen05 kernels)."""
+    _check(lib().moe_set_cold_expert_tokens(int(max_tokens)), "moe_set_cold_expert_tokens")
 
 
 def moe_check_status(workspace, stream=None):

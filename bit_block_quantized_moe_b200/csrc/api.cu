@@ -357,6 +357,12 @@ moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after) {
   return MOE_OK;
 }
 
+moe_status moe_set_cold_expert_tokens(int32_t max_tokens) {
+  if (max_tokens < 0 || max_tokens > 64) return MOE_ERR_ARG;
+  set_cold_expert_tokens(max_tokens);
+  return MOE_OK;
+}
+
 moe_status moe_check_status(void *workspace, moe_stream_t stream) {
   if (!workspace) return MOE_ERR_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -54,6 +54,10 @@ cudaError_t launch_experts(const moe_dims &d, const PackedGeom &G, const uint8_t
                            const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
 // Tokens per tcgen05 prefill work item for T tokens (64, or 128 once an expert averages 64 tokens).
 int tc_item_tokens(const moe_dims &d, int T);
+// In a prefill chunk (T > 8), experts with at most this many tokens run on the register-dequant expert
+// kernels instead of the tcgen05 ones (0: none).
+int cold_expert_tokens(const moe_dims &d, int T);
+void set_cold_expert_tokens(int n);
 cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                               const uint16_t *x, int T, const Workspace &ws, cudaStream_t s);
 cudaError_t launch_combine(const moe_dims &d, int T, const Workspace &ws, uint16_t *out, cudaStream_t s);

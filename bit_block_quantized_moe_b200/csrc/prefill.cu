@@ -33,6 +33,8 @@
 // The issuing thread of the MMAs is the pipeline's pace: everything it waits
 // on is taken off its path.  Accumulators are double-buffered so the epilogue
 // of one item overlaps the MMAs of the next.  Every wait is bounded (sync.cuh).
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -41,6 +43,7 @@ namespace moe {
 namespace {
 
 constexpr int kTileUnits = 8;      // 16-row units per 128-row M tile
+
 constexpr int kWarpProducer = 0, kWarpMMA = 1, kWarpDequant0 = 2, kNumDequant = 16, kWarpEpi0 = 18, kNumEpi = 4;
 constexpr int kThreadsTC = (kWarpEpi0 + kNumEpi) * 32;  // 704
 constexpr uint32_t kTmemCols = 512;
@@ -474,8 +477,28 @@ int tc_item_tokens(const moe_dims &d, int T) {
   return (long long)T * d.top_k >= 64LL * d.n_experts ? CfgMany::kMaxN : CfgFew::kMaxN;
 }
 
+// Experts of a prefill chunk with at most this many tokens go to the register-dequant kernels (one 8-token
+// item each), the rest to the tcgen05 kernels; set per host thread by moe_set_cold_expert_tokens.  0 (none) by
+// default: on B200 the tcgen05 path was faster for every expert, down to one token.
+static thread_local int g_cold_expert_tokens = 0;
+
+void set_cold_expert_tokens(int n) { g_cold_expert_tokens = n; }
+
+int cold_expert_tokens(const moe_dims &d, int T) {
+  (void)d;
+  (void)T;
+  return g_cold_expert_tokens;
+}
+
 cudaError_t launch_tc_experts(const moe_dims &d, const PackedGeom &G, const uint8_t *experts, const uint8_t *shared,
                               const uint16_t *x, int T, const Workspace &ws, cudaStream_t s) {
+  const int cold = cold_expert_tokens(d, T);
+  if (cold > 0) {  // the cold experts' items on the register-dequant kernels first
+    Workspace wc = ws;  // grid sized by the cold list's bound: at most ceil(cold / 8) items per expert
+    wc.max_items = (int)std::min<long long>(ws.max_items, (long long)d.n_experts * ((cold + 7) / 8));
+    const cudaError_t e0 = launch_experts(d, G, experts, shared, x, T, wc, s);
+    if (e0 != cudaSuccess) return e0;
+  }
   const int P = T * d.top_k + T;  // sorted positions (routed + shared)
   trace_mark(MOE_KERNEL_GATHER, false, s);
   gather_rows_kernel<<<(unsigned)(((long long)P * 32 + 255) / 256), 256, 0, s>>>(x, ws.sorted_tok, P, G.H, ws.xs);

@@ -312,9 +312,11 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const float *Wr, 
 
 // One CTA of 1024 threads: per expert (one warp each, in turn) the popcount
 // prefix of its membership words and its count; then a block-wide exclusive
-// scan gives the offsets and the starts of each expert's work items (tiles of
-// 8 tokens for the register-dequant path, 64 for the tcgen05 path); the shared
-// expert's items follow the routed ones.
+// scan gives the offsets and the starts of each expert's work items: tiles of
+// 8 tokens for the register-dequant path (experts with at most cold_max
+// tokens) and of tc_n tokens for the tcgen05 path (the other experts); the
+// shared expert's items follow the routed ones, on the register-dequant list
+// when shared_cold, else on the tcgen05 list.
 constexpr int kScanThreads = 1024;
 
 __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int &total) {
@@ -368,7 +370,8 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_wscan_kernel(const uint
 __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int T, int k,
                                                                      const int32_t *__restrict__ counts,
                                                                      int32_t *offsets, int4 *items, uint32_t *n_items,
-                                                                     int4 *tc_items, uint32_t *n_tc_items, int tc_n) {
+                                                                     int4 *tc_items, uint32_t *n_tc_items, int tc_n,
+                                                                     int cold_max, int shared_cold) {
   __shared__ int warp_sums[33];
   // thread i owns experts [i * per, (i + 1) * per)
   const int per = (E + kScanThreads - 1) / kScanThreads;
@@ -377,8 +380,8 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int 
   for (int i = eb; i < ee; ++i) {
     const int c = counts[i];
     my_cnt += c;
-    my_items += (c + 7) >> 3;
-    my_tc += (c + tc_n - 1) / tc_n;
+    if (c <= cold_max) my_items += (c + 7) >> 3;
+    else my_tc += (c + tc_n - 1) / tc_n;
   }
   int tot_cnt, tot_items, tot_tc;
   int pos = block_exclusive_scan(my_cnt, warp_sums, tot_cnt);
@@ -387,12 +390,14 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(int E, int 
   for (int i = eb; i < ee; ++i) {
     const int c = counts[i];
     offsets[i] = pos;
-    for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
-    for (int j = 0; j < c; j += tc_n) tc_items[itc++] = make_int4(i, pos + j, min(tc_n, c - j), 0);
+    if (c <= cold_max)
+      for (int j = 0; j < c; j += 8) items[it++] = make_int4(i, pos + j, min(8, c - j), 0);
+    else
+      for (int j = 0; j < c; j += tc_n) tc_items[itc++] = make_int4(i, pos + j, min(tc_n, c - j), 0);
     pos += c;
   }
   // the shared expert's items follow the routed ones
-  const int shared_items = (T + 7) >> 3, shared_tc = (T + tc_n - 1) / tc_n;
+  const int shared_items = shared_cold ? (T + 7) >> 3 : 0, shared_tc = shared_cold ? 0 : (T + tc_n - 1) / tc_n;
   for (int i = threadIdx.x; i < shared_items; i += blockDim.x)
     items[tot_items + i] = make_int4(E, T * k + 8 * i, min(8, T - 8 * i), 0);
   for (int i = threadIdx.x; i < shared_tc; i += blockDim.x)
@@ -463,8 +468,12 @@ cudaError_t launch_dispatch(const moe_dims &d, int T, const Workspace &ws, cudaS
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, false, s);
   const int wthreads = std::min(kScanThreads, (ws.words + 31) & ~31);
   dispatch_wscan_kernel<<<E, wthreads, 0, s>>>(ws.bitmap, ws.words, ws.wprefix, ws.counts);
+  // few tokens: every expert on the register-dequant list; a prefill chunk: experts with at most
+  // cold_expert_tokens(T) tokens there, the rest and the shared expert on the tcgen05 list
+  const bool small = T <= 8;
   dispatch_scan_kernel<<<1, kScanThreads, 0, s>>>(E, T, k, ws.counts, ws.offsets, ws.items, ws.n_items, ws.tc_items,
-                                                  ws.n_tc_items, ws.tc_item_tokens > 0 ? ws.tc_item_tokens : 64);
+                                                  ws.n_tc_items, ws.tc_item_tokens > 0 ? ws.tc_item_tokens : 64,
+                                                  small ? 0x7fffffff : cold_expert_tokens(d, T), small ? 1 : 0);
   trace_mark(MOE_KERNEL_DISPATCH_SCAN, true, s);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;

@@ -275,6 +275,20 @@ enum {
 };
 moe_status moe_trace_kernel(int32_t kernel_id, void *before, void *after);
 
+/* ---- per-expert kernel choice in a prefill chunk ---------------------------------------
+ * Verify windows hold a few tokens (devlabs page, section 1; Strata tuning
+ * page, sections 5 and 8: --spec 4/6/8), and in a prefill chunk with a skewed
+ * router many experts get only a few tokens.  In a chunk of T > 8 tokens,
+ * experts routed at most max_tokens tokens run on the register-dequant expert
+ * kernels (8-token items) and the others, with the shared expert, on the
+ * tcgen05 kernels.  The setting is per host thread; 0 (the default) sends
+ * every expert to the tcgen05 kernels.  Measured on B200 (hidden 2048, 512
+ * experts, Zipf router): any max_tokens > 0 was slower at every T from 16 to
+ * 1024, because one tcgen05 work item costs less than one register-dequant
+ * item even for a one-token expert; keep 0 unless measurement on another shape
+ * says otherwise.  0 <= max_tokens <= 64, else MOE_ERR_ARG. */
+moe_status moe_set_cold_expert_tokens(int32_t max_tokens);
+
 /* ---- status ----------------------------------------------------------------------
  * Blocking host call: waits for `stream`, reads and clears the sticky device
  * status word in `workspace`; MOE_OK, MOE_ERR_DEVICE or MOE_ERR_TIMEOUT. */

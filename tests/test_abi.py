@@ -82,6 +82,8 @@ def test_host_checks_before_launch(lib):
     assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 4, 0x2000, 0x3000, None, 0x5000, 0x10000, ws, None) == 1
     assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 4, 0x2000, 0x3000, 0x4000, 0x5000, 0x10004, ws, None) == 2
     assert lib.moe_dispatch(ctypes.byref(d), 0x1000, 9, 0x2000, 0x3000, 0x4000, 0x5000, 0x10000, 16, None) == 3
+    assert lib.moe_set_cold_expert_tokens(-1) == 1 and lib.moe_set_cold_expert_tokens(65) == 1
+    assert lib.moe_set_cold_expert_tokens(8) == 0 and lib.moe_set_cold_expert_tokens(0) == 0
     assert lib.moe_rmsnorm_residual(None, None, None, 0, 256, 1e-6, None) == 0
     assert lib.moe_rmsnorm_residual(None, None, None, 4, 256, 1e-6, None) == 1
 

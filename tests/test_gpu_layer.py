@@ -125,6 +125,31 @@ def test_prefill_ragged_and_cold_tail():
     check_layer(cfg, w, x, y, idx, wts)
 
 
+@pytest.mark.parametrize("cold", [0, 8])
+def test_verify_windows_and_cold_tail_per_expert_kernels(cold):
+    """Wider verify windows (T = 16, 32, 64 tokens: --spec 4/6/8 windows, Strata tuning page sections 5 and 8) and
+    the cold-tail router (many experts with 1-2 tokens), every token against the oracle, with every expert on the
+    tcgen05 kernels (cold = 0, the default) and with experts of at most 8 tokens on the register-dequant kernels
+    (cold = 8, moe_set_cold_expert_tokens)."""
+    from bit_block_quantized_moe_b200 import moe_set_cold_expert_tokens
+
+    moe_set_cold_expert_tokens(cold)
+    try:
+        for bias, Ts in (("zipf", (16, 32, 64)), ("zipf_cold", (133, 1024))):
+            cfg = MoeConfig("windows", 2048, 512, 512, 10, 64, bias)
+            L, w = build_layer(cfg, seed=2)
+            for T in Ts:
+                x = make_x(T, 2048, seed=60 + T)
+                y, idx, wts = gpu_forward(L, x)
+                err, l2, flagged = check_layer(cfg, w, x, y, idx, wts)
+                counts = np.bincount(idx.ravel(), minlength=512)
+                print(f"cold={cold} {bias} T={T}: max-rel {err:.3e} relL2 {l2:.3e} flagged {len(flagged)}; experts "
+                      f"with <= 8 tokens: {int(((counts > 0) & (counts <= 8)).sum())}")
+            del L
+    finally:
+        moe_set_cold_expert_tokens(0)
+
+
 def test_route_entry_point(full):
     L, w = full
     cfg = CONFIGS["prefill"]
