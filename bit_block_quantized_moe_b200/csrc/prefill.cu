@@ -166,8 +166,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
   const uint32_t tbase = B.tmem;
 
   if (warp == kWarpProducer) {
-    // The whole warp runs the loop; one elected lane issues the copies.
-    int cnt = 0;
+    // The whole warp runs the loop; one elected lane issues the copies.  After a wait gives up no further
+    // copy is issued, so the copies in flight are those of counts [issued - kStages, issued).
+    int cnt = 0, issued = 0;
+    bool live = true;
     for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
       const int4 it = a.items[w / a.mgroups];
       const int mt0 = (w % a.mgroups) * kMT;
@@ -177,7 +179,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
       const int ae = it.x == a.E ? 0 : it.x;
       for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
         const int s = cnt % kStages;
-        if (!waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) continue;
+        if (live && !waitb(&B.empty[s], ((cnt / kStages) & 1) ^ 1, B, a.status)) live = false;
+        if (!live) continue;
+        issued = cnt + 1;
         if (elect_one()) {
           uint8_t *st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&B.full[s], (uint32_t)(kABytes + 2 * nrows * 128));
@@ -189,8 +193,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
         __syncwarp();
       }
     }
-    // every copy issued must land before the CTA exits
-    for (int c2 = max(0, cnt - kStages); c2 < cnt; ++c2) waitb(&B.full[c2 % kStages], (c2 / kStages) & 1, B, a.status);
+    // Every copy issued must land before the CTA exits, also after an abort: a bounded wait of its own
+    // (the shared abort flag would end it at once), the phase of count c2 being the last one its stage had.
+    for (int c2 = max(0, issued - kStages); c2 < issued; ++c2)
+      if (!mbar_wait(&B.full[c2 % kStages], (c2 / kStages) & 1)) set_status(a.status, kStatusTimeout);
   } else if (warp == kWarpMMA) {
     // The whole warp runs the loop on warp-uniform values; one elected lane issues the MMAs and commits.
     int cnt = 0, dcnt = 0;

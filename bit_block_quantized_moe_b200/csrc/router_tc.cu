@@ -114,13 +114,17 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   const uint32_t tbase = B.tmem;
 
   if (warp == 0) {
-    // The whole warp runs the loop on warp-uniform values; one elected lane issues the copies.
-    int cnt = 0;
+    // The whole warp runs the loop on warp-uniform values; one elected lane issues the copies.  After a wait
+    // gives up no further copy is issued, so the copies in flight are those of counts [issued - stages, issued).
+    int cnt = 0, issued = 0;
+    bool live = true;
     for (int u = blockIdx.x; u < a.n_units; u += gridDim.x) {
       const int ks = u % a.ks, tile = u / a.ks, et = tile % a.n_et, tt = tile / a.n_et;
       for (int c = 0; c < kper / kRtK; ++c, ++cnt) {
         const int s = cnt % kRtStages;
-        if (!rt_wait(&B.empty[s], ((cnt / kRtStages) & 1) ^ 1, B, a.status)) continue;
+        if (live && !rt_wait(&B.empty[s], ((cnt / kRtStages) & 1) ^ 1, B, a.status)) live = false;
+        if (!live) continue;
+        issued = cnt + 1;
         if (elect_one()) {
           uint8_t *st = smem + s * kRtStageBytes;
           mbar_arrive_expect_tx(&B.full[s], (uint32_t)kRtStageBytes);
@@ -131,9 +135,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         __syncwarp();
       }
     }
-    // every copy issued must land before the CTA exits
-    for (int c2 = max(0, cnt - kRtStages); c2 < cnt; ++c2)
-      rt_wait(&B.full[c2 % kRtStages], (c2 / kRtStages) & 1, B, a.status);
+    // Every copy issued must land before the CTA exits, also after an abort: a bounded wait of its own
+    // (the shared abort flag would end it at once), the phase of count c2 being the last one its stage had.
+    for (int c2 = max(0, issued - kRtStages); c2 < issued; ++c2)
+      if (!mbar_wait(&B.full[c2 % kRtStages], (c2 / kRtStages) & 1)) set_status(a.status, kStatusTimeout);
   } else if (warp == 1) {
     // The whole warp runs the loop on warp-uniform values; one elected lane issues the MMAs and commits (a
     // lane-0-only loop issues them about 20% slower).
