@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       const int r = r0 + warp / kRouterParts, q = warp % kRouterParts;
       if (r < n_rrows) {
         float acc[8];
-        router_part<true>(xs, xstride, T, wr_s + (size_t)r * H, H, q, lane, acc);
+        router_part_any<true>(xs, xstride, T, wr_s + (size_t)r * H, H, q, lane, acc);
         if (lane == 0) {
 #pragma unroll
           for (int t = 0; t < 8; ++t) rpart[((r - r0) * kMaxTok + t) * kRouterParts + q] = acc[t];
@@ -295,7 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       int e;
       float wt;
       uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
-      if (E <= 512)
+      if (E == 512)
+        warp_topk_fast<16, true, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+      else if (E < 512)
         warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
       else
         warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);

@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(64) router_logits_small_kernel(const uint16_t 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x;
   float acc[8];
-  router_part<false>(x, H, T, Wr + (size_t)e * H, H, warp, lane, acc);
+  router_part_any<false>(x, H, T, Wr + (size_t)e * H, H, warp, lane, acc);
   if (lane == 0) {
 #pragma unroll
     for (int t = 0; t < 8; ++t) part[t][warp] = acc[t];
@@ -259,7 +259,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
   float wt;
   int e;
   const float *row = logits + (size_t)t * E;
-  if (E <= 512)
+  if (E == 512)
+    warp_topk_fast<16, false, true>(row, E, k, lane, scratch[threadIdx.x >> 5], e, wt);
+  else if (E < 512)
     warp_topk_fast<16>(row, E, k, lane, scratch[threadIdx.x >> 5], e, wt);
   else if (E <= 1024)
     warp_topk_fast<32>(row, E, k, lane, scratch[threadIdx.x >> 5], e, wt);

@@ -10,11 +10,15 @@ namespace moe {
 // half h is summed by one warp: lane l accumulates k = h*H/2 + 4l + 128 i in
 // order, then a butterfly sum.  The logit is (p0 + p1) + b.  Both the routing
 // kernel and the fused decode kernel use exactly this order, so they take
-// identical routing decisions.
+// identical routing decisions.  kT is the token count when it is fixed at
+// compile time (0: T at run time); the arithmetic is the same either way, but a
+// run-time T leaves all 8 token slots in the code behind predicates, about
+// twice the cycles for T = 3 on B200 (router_part_any picks the instance).
 constexpr int kRouterParts = 2;
-template <bool kWrShared>
-__device__ __forceinline__ void router_part(const uint16_t *x, int xstride, int T, const float *wrow, int H,
+template <bool kWrShared, int kT = 0>
+__device__ __forceinline__ void router_part(const uint16_t *x, int xstride, int T_, const float *wrow, int H,
                                             int part, int lane, float (&acc)[8]) {
+  const int T = kT ? kT : T_;
 #pragma unroll
   for (int t = 0; t < 8; ++t) acc[t] = 0.f;
   const int kq = H / kRouterParts;
@@ -38,8 +42,25 @@ __device__ __forceinline__ void router_part(const uint16_t *x, int xstride, int 
   }
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
+    if (t < T) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+      for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    }
+  }
+}
+
+template <bool kWrShared>
+__device__ __forceinline__ void router_part_any(const uint16_t *x, int xstride, int T, const float *wrow, int H,
+                                                int part, int lane, float (&acc)[8]) {
+  switch (T) {
+    case 1: router_part<kWrShared, 1>(x, xstride, T, wrow, H, part, lane, acc); break;
+    case 2: router_part<kWrShared, 2>(x, xstride, T, wrow, H, part, lane, acc); break;
+    case 3: router_part<kWrShared, 3>(x, xstride, T, wrow, H, part, lane, acc); break;
+    case 4: router_part<kWrShared, 4>(x, xstride, T, wrow, H, part, lane, acc); break;
+    case 5: router_part<kWrShared, 5>(x, xstride, T, wrow, H, part, lane, acc); break;
+    case 6: router_part<kWrShared, 6>(x, xstride, T, wrow, H, part, lane, acc); break;
+    case 7: router_part<kWrShared, 7>(x, xstride, T, wrow, H, part, lane, acc); break;
+    default: router_part<kWrShared, 8>(x, xstride, T, wrow, H, part, lane, acc); break;
   }
 }
 
@@ -189,7 +210,9 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // more than 32 values pass.  Few dependent steps: shared-memory broadcasts
 // instead of shuffle chains.  `scratch` is 64 uint64 of shared memory private
 // to the warp.  Same selection and softmax as warp_topk, hence the same result.
-template <int NPL, bool kSmem = false>
+// kFull: E == 32 * NPL, so every lane loads all its values with no bounds test
+// (the run-time test around each load costs about 1.7k cycles per call on B200).
+template <int NPL, bool kSmem = false, bool kFull = false>
 __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, int lane, uint64_t *scratch,
                                                int &e_out, float &w_out) {
   uint32_t kv[NPL];
@@ -197,7 +220,7 @@ __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, i
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
     const int e = lane + 32 * j;
-    kv[j] = e < E ? float_key(load_logit<kSmem>(row, e)) : 0u;
+    kv[j] = (kFull || e < E) ? float_key(load_logit<kSmem>(row, e)) : 0u;
     mk = kv[j] > mk ? kv[j] : mk;
   }
   uint32_t *lmax = reinterpret_cast<uint32_t *>(scratch + 32);  // 32 lane maxima
