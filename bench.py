@@ -604,7 +604,8 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src, sampler):
     gu_ms = traced_kernel_ms(step, min(K, 8), M.MOE_KERNEL["gate_up"], stream)
     dn_ms = traced_kernel_ms(step, min(K, 8), M.MOE_KERNEL["down"], stream)
     gu_flops = (T * cfg.top_k + T) * 4 * H * cfg.inter
-    gu_bytes = (touched + 1) * EXPERT_BYTES * 2 / 3 + (T * cfg.top_k + T) * H * 2  # gate/up sections + token rows
+    # gate/up sections + token rows read, h (bf16) written
+    gu_bytes = (touched + 1) * EXPERT_BYTES * 2 / 3 + (T * cfg.top_k + T) * H * 2 + (T * cfg.top_k + T) * cfg.inter * 2
     traffic, traffic_note = profiled_traffic(PREFILL_PROFILE, PREFILL_SOURCES, "dram bytes per launch (gate/up)")
     M.moe_check_status(ws)
     return {
