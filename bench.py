@@ -250,8 +250,10 @@ def capture(fn, n_steps, stream, first=0):
     return g
 
 
-def time_graph_steps(fn, K, W, stream, world, chunk=240, win=None):
-    """Warm up W steps, then time exactly K steps (graphs of <= chunk steps); returns seconds (max over ranks)."""
+def time_graph_steps(fn, K, W, stream, world, chunk=240, win=None, dist=None):
+    """Warm up W steps, then time exactly K steps (graphs of <= chunk steps); returns seconds (max over ranks).
+    With `dist` (a dict), an event after every replay also gives the per-step time of each replay: its median,
+    p10, p90 (ms per step, this rank) and the number of replays are stored there."""
     import torch
 
     gw = capture(fn, max(1, min(W, chunk)), stream) if W > 0 else None
@@ -270,17 +272,33 @@ def time_graph_steps(fn, K, W, stream, world, chunk=240, win=None):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    marks = []  # (event after a replay, steps in it)
     with (win if win is not None else _Null()), torch.cuda.stream(stream):
         start.record(stream)
         for _ in range(full):
             g_full.replay()
+            if dist is not None:
+                marks.append((torch.cuda.Event(enable_timing=True), chunk))
+                marks[-1][0].record(stream)
         if g_rem is not None:
             g_rem.replay()
+            if dist is not None:
+                marks.append((torch.cuda.Event(enable_timing=True), rem))
+                marks[-1][0].record(stream)
         end.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     secs = start.elapsed_time(end) / 1e3
+    if dist is not None and marks:
+        import numpy as np
+        per, prev = [], start
+        for ev, n in marks:
+            per.append(prev.elapsed_time(ev) / n)
+            prev = ev
+        q = np.percentile(np.array(per), [10, 50, 90])
+        dist.update({"ms_per_step_p10": float(q[0]), "ms_per_step_median": float(q[1]),
+                     "ms_per_step_p90": float(q[2]), "replays": len(per)})
     del gw, g_full, g_rem
     return max_over_ranks(secs, world)
 
@@ -433,11 +451,13 @@ def run_decode(args, cfg, sets, routers, dims, T, K, W, world, rank, dev, stream
         check = {k: sum(c[k] for c in ci) for k in ci[0]}
 
     win = sampler.window(f"decode T={T}") if sampler is not None else None
-    secs = time_graph_steps(step, K, W, stream, world, win=win)
+    dist = {}
+    secs = time_graph_steps(step, K, W, stream, world, win=win, dist=dist)
     ms_per_step = secs * 1e3 / K
     avg_touched = float(np.mean([touched[(i % n_sets % n_distinct) * n_slots + (i % n_slots)] for i in range(K)]))
     bytes_ = layer_bytes(avg_touched, cfg.n_experts, H, T)
-    out = {"T": T, "ms_per_step": ms_per_step, "value": world * T * K / secs, "unit": "tokens/s", "steps": K,
+    out = {"T": T, "ms_per_step": ms_per_step, "step_dist": dist, "value": world * T * K / secs, "unit": "tokens/s",
+           "steps": K,
            "touched_experts_per_step": avg_touched, "bytes_per_step": bytes_,
            "achieved_gbs": bytes_ / (ms_per_step * 1e-3) / 1e9,
            "frac_of_measured_hbm": bytes_ / (ms_per_step * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
@@ -544,6 +564,7 @@ def run_ours(args, world, rank, local):
         },
         "routing_check": d["routing_check"],
         "e2e": d["e2e"],
+        "step_dist": d["step_dist"],
         "gpu_launches": K,
     }
 
@@ -592,7 +613,8 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src, sampler):
     check = routing_check(xs_np[0], routers[0][0], routers[0][1], idx_np[0], cfg.top_k) if rank == 0 else None
     K = args.prefill_steps
     win = sampler.window("prefill T=1024") if sampler is not None else None
-    secs = time_graph_steps(step, K, 3, stream, world, chunk=20, win=win)
+    dist = {}
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=4, win=win, dist=dist)
     ms = secs * 1e3 / K
     bytes_ = layer_bytes(touched, cfg.n_experts, H, T)
     flops = layer_flops(T, cfg.top_k, H, cfg.inter, cfg.n_experts)
@@ -612,6 +634,7 @@ def run_prefill(args, world, rank, dev, stream, peaks, peak_src, sampler):
         "value": world * T * K / secs,
         "unit": "tokens/s",
         "ms_per_step": ms,
+        "step_dist": dist,
         "steps": K,
         "workload": "prefill chunk: T=1024, Zipf(s=1.1) router bias (hottest expert ~100 slots), same layer dims",
         "touched_experts": touched,
@@ -663,7 +686,8 @@ def run_32k(args, world, rank, dev, stream, peaks, peak_src, sampler, K_dec, W_d
 
     K = 4
     win = sampler.window("prefill T=32768") if sampler is not None else None
-    secs = time_graph_steps(step, K, 3, stream, world, chunk=K, win=win)
+    dist = {}
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=1, win=win, dist=dist)
     ms_layer = secs * 1e3 / (K * L)
     bytes_ = sum(layer_bytes(t, cfg.n_experts, H, T) for t in touched) / L
     flops = layer_flops(T, cfg.top_k, H, cfg.inter, cfg.n_experts)
@@ -673,7 +697,7 @@ def run_32k(args, world, rank, dev, stream, peaks, peak_src, sampler, K_dec, W_d
     M.moe_check_status(ws)
     big = {
         "value": world * T * K * L / secs, "unit": "tokens/s (layer passes)", "ms_per_layer": ms_layer,
-        "ms_per_step": ms_layer * L, "layers_per_step": L, "steps": K,
+        "ms_per_step": ms_layer * L, "step_dist": dist, "layers_per_step": L, "steps": K,
         "workload": "4 full-size layers (hidden 2048, 512 experts top-10 + shared, inter 512), T=32768, Zipf router; "
                     "each layer reads the same x",
         "bytes_per_layer": bytes_, "flops_per_layer": flops,
@@ -686,7 +710,7 @@ def run_32k(args, world, rank, dev, stream, peaks, peak_src, sampler, K_dec, W_d
     for Td in (1, 2, 3):
         r = run_decode(args, cfg, sets, routers, dims, Td, min(K_dec, 2000), W_dec, world, rank, dev, stream, peaks,
                        peak_src, sampler)
-        sweep[f"T{Td}"] = {k: r[k] for k in ("value", "unit", "ms_per_step", "touched_experts_per_step",
+        sweep[f"T{Td}"] = {k: r[k] for k in ("value", "unit", "ms_per_step", "step_dist", "touched_experts_per_step",
                                              "bytes_per_step", "achieved_gbs", "frac_of_measured_hbm",
                                              "frac_of_8tbs", "routing_check")}
     sweep["workload"] = "decode T=1,2,3 on 24 rotating copies of the four Zipf-routed 32768-token-case layers"
@@ -744,7 +768,8 @@ def run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler):
     torch.cuda.synchronize()
     K = max(1, min(args.steps, 5))
     win = sampler.window("stack 48 x T=1024") if sampler is not None else None
-    secs = time_graph_steps(step, K, 3, stream, world, chunk=1, win=win)
+    dist = {}
+    secs = time_graph_steps(step, K, 3, stream, world, chunk=1, win=win, dist=dist)
     ms = secs * 1e3 / K
     secs_u = time_graph_steps(step_unfused, K, 3, stream, world, chunk=1)
     ms_u = secs_u * 1e3 / K
@@ -757,7 +782,7 @@ def run_stack(args, world, rank, dev, stream, peaks, peak_src, sampler):
     del sets
     torch.cuda.empty_cache()
     return {
-        "value": world * T * K / secs, "unit": "tokens/s (through all 48 layers)", "ms_per_step": ms,
+        "value": world * T * K / secs, "unit": "tokens/s (through all 48 layers)", "ms_per_step": ms, "step_dist": dist,
         "ms_per_layer": ms / L, "steps": K, "layers": L,
         "workload": "48 full-size layers (hidden 2048, 512 experts top-10 + shared, inter 512), T=1024, Zipf router, "
                     "RMSNorm eps 1e-6 + residual between layers, independent seeded weights per layer (24 GB)",

@@ -10,8 +10,9 @@
 //        CTA prepares its token rows as the MMA B operand (block correction
 //        sums, the (4c+2, 4c+3) pairs scaled by 1/4) --
 //  B  All logits into shared memory; one warp per token selects the top-k
-//     (threshold + rank) and the CTA builds the same sorted list of touched
-//     experts plus the shared expert as every other CTA.
+//     (threshold + rank) and marks its experts in a bit map (the tables were
+//     cleared while waiting on the barrier); one warp builds the same sorted
+//     list of touched experts plus the shared expert as every other CTA.
 //  C  Work lists, expert-major, cut into equal contiguous ranges per CTA:
 //     gate/up units (expert, 8 intermediate rows) and down stages (expert, two
 //     16-row units).  Stage s belongs to warp s % 14, which copies it into its
@@ -282,6 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     const bool leader = tid == kConsumers - 1;
     const uint64_t bar_target = grid_arrive(a.gbar, kBarConsumers, kConsumers, leader);
     prep_rows(xs, xstride, H, T, corr, tid);
+    // the touched-expert tables start empty (filled once the top-k is known)
+    for (int i = tid; i < kMaxEntries * kMaxTok; i += kConsumers) {
+      tokj[i] = -1;
+      tokw[i] = 0.f;
+    }
+    if (tid < kMaxE / 32) bitmap[tid] = 0u;
     grid_wait(a.gbar, bar_target, kBarConsumers, kConsumers, leader, a.status, &misc[2]);
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
@@ -304,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       if (lane < K) {
         sel_idx[warp * K + lane] = e;
         sel_w[warp * K + lane] = wt;
+        atomicOr(&bitmap[e >> 5], 1u << (e & 31));
         if (blockIdx.x == 0 && a.idx_out) {
           a.idx_out[warp * K + lane] = e;
           a.w_out[warp * K + lane] = wt;
@@ -312,10 +320,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     }
     named_bar(kBarConsumers, kConsumers);
     if (warp == 0) {
-      bitmap[lane] = 0u;
-      __syncwarp();
-      for (int i = lane; i < T * K; i += 32) atomicOr(&bitmap[sel_idx[i] >> 5], 1u << (sel_idx[i] & 31));
-      __syncwarp();
       const uint32_t word = bitmap[lane];
       const uint32_t cnt = __popc(word);
       uint32_t incl = cnt;
@@ -333,10 +337,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         ent[r] = lane * 32 + b;
       }
       const int U = __shfl_sync(0xffffffffu, (int)incl, 31);
-      for (int i = lane; i < (U + 1) * kMaxTok; i += 32) {
-        tokj[i] = -1;
-        tokw[i] = 0.f;
-      }
       __syncwarp();
       for (int i = lane; i < T * K; i += 32) {
         const int t = i / K, j = i % K, e = sel_idx[i];
