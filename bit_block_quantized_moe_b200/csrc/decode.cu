@@ -9,7 +9,7 @@
 //     -- grid barrier: all logits written.  Between arriving and waiting the
 //        CTA prepares its token rows as the MMA B operand (block correction
 //        sums, the (4c+2, 4c+3) pairs scaled by 1/4) --
-//  B  All logits into shared memory; one warp per token selects the top-k
+//  B  One warp per token reads its logits from L2 and selects the top-k
 //     (threshold + rank) and marks its experts in a bit map (the tables were
 //     cleared while waiting on the barrier); one warp builds the same sorted
 //     list of touched experts plus the shared expert as every other CTA.
@@ -292,22 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     grid_wait(a.gbar, bar_target, kBarConsumers, kConsumers, leader, a.status, &misc[2]);
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
-    // All logits into shared memory first (one coalesced pass through L2), then one warp per token.
-    float *lg = reinterpret_cast<float *>(ring);  // the ring is free until the stages start
-    for (int i = tid; i < T * E / 4; i += kConsumers)
-      reinterpret_cast<float4 *>(lg)[i] = ldg_cg_f4(a.logits + 4 * (size_t)i);
-    for (int i = (T * E / 4) * 4 + tid; i < T * E; i += kConsumers) lg[i] = __ldcg(a.logits + i);
-    named_bar(kBarConsumers, kConsumers);
+    // One warp per token reads its token's logits straight from L2 (other CTAs wrote them).
     if (warp < T) {
       int e;
       float wt;
       uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
+      const float *row = a.logits + (size_t)warp * E;
       if (E == 512)
-        warp_topk_fast<16, true, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+        warp_topk_fast<16, false, true>(row, E, K, lane, scratch, e, wt);
       else if (E < 512)
-        warp_topk_fast<16, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+        warp_topk_fast<16, false>(row, E, K, lane, scratch, e, wt);
       else
-        warp_topk_fast<32, true>(lg + (size_t)warp * E, E, K, lane, scratch, e, wt);
+        warp_topk_fast<32, false>(row, E, K, lane, scratch, e, wt);
       if (lane < K) {
         sel_idx[warp * K + lane] = e;
         sel_w[warp * K + lane] = wt;
