@@ -9,10 +9,12 @@
 //     -- grid barrier: all logits written.  Between arriving and waiting the
 //        CTA prepares its token rows as the MMA B operand (block correction
 //        sums, the (4c+2, 4c+3) pairs scaled by 1/4) --
-//  B  One warp per token reads its logits from L2 and selects the top-k
+//  B  One warp per token reads its logits from L2, selects the top-k
 //     (threshold + rank) and marks its experts in a bit map (the tables were
-//     cleared while waiting on the barrier); one warp builds the same sorted
-//     list of touched experts plus the shared expert as every other CTA.
+//     cleared while waiting on the barrier).  Then a spare warp builds the
+//     same sorted list of touched experts plus the shared expert as every
+//     other CTA, while the token warps compute their weights (softmax over
+//     their winners) and fill their table entries.
 //  C  Work lists, expert-major, cut into equal contiguous ranges per CTA:
 //     gate/up units (expert, 8 intermediate rows) and down stages (expert, two
 //     16-row units).  Stage s belongs to warp s % 14, which copies it into its
@@ -78,7 +80,7 @@ struct DecodeArgs {
 };
 
 struct SmemLayout {
-  uint32_t xs, corr, hcorr, rpart, red, sel_idx, sel_w, bitmap, wpre, ent, tokj, tokw, misc, ring, total;
+  uint32_t xs, corr, hcorr, rpart, red, bitmap, ent, tokj, tokw, misc, ring, total;
 };
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -97,13 +99,7 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   o = align_to(o, 16);
   L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
   o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
-  L.sel_idx = o;
-  o += kMaxSel * 4;
-  L.sel_w = o;
-  o += kMaxSel * 4;
   L.bitmap = o;
-  o += (kMaxE / 32) * 4;
-  L.wpre = o;
   o += (kMaxE / 32) * 4;
   L.ent = o;
   o = align_to(o + kMaxEntries * 4, 16);
@@ -203,10 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   float *hcorr = reinterpret_cast<float *>(smem + L.hcorr);
   float *rpart = reinterpret_cast<float *>(smem + L.rpart);
   float *red = reinterpret_cast<float *>(smem + L.red);
-  int *sel_idx = reinterpret_cast<int *>(smem + L.sel_idx);
-  float *sel_w = reinterpret_cast<float *>(smem + L.sel_w);
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + L.bitmap);
-  uint32_t *wpre = reinterpret_cast<uint32_t *>(smem + L.wpre);
   int *ent = reinterpret_cast<int *>(smem + L.ent);
   int8_t *tokj = reinterpret_cast<int8_t *>(smem + L.tokj);
   float *tokw = reinterpret_cast<float *>(smem + L.tokw);
@@ -293,29 +286,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
 
     // ---------------- phase B: top-k and the touched-expert list ----------------
     // One warp per token reads its token's logits straight from L2 (other CTAs wrote them).
+    int e = 0;
+    float lv = 0.f;
     if (warp < T) {
-      int e;
-      float wt;
       uint64_t *scratch = reinterpret_cast<uint64_t *>(red) + warp * 64;
       const float *row = a.logits + (size_t)warp * E;
       if (E == 512)
-        warp_topk_fast<16, false, true>(row, E, K, lane, scratch, e, wt);
+        warp_topk_fast_sel<16, false, true>(row, E, K, lane, scratch, e, lv);
       else if (E < 512)
-        warp_topk_fast<16, false>(row, E, K, lane, scratch, e, wt);
+        warp_topk_fast_sel<16, false>(row, E, K, lane, scratch, e, lv);
       else
-        warp_topk_fast<32, false>(row, E, K, lane, scratch, e, wt);
+        warp_topk_fast_sel<32, false>(row, E, K, lane, scratch, e, lv);
+      if (lane < K) atomicOr(&bitmap[e >> 5], 1u << (e & 31));
+    }
+    named_bar(kBarConsumers, kConsumers);  // every selected expert is in the bit map
+    if (warp < T) {
+      // While a spare warp builds the list: the token's weights (fp32 softmax over its winners) and its
+      // table entries, each lane ranking its expert among the touched ones from the bit map.
+      const float wt = topk_softmax(lv, lane, K);
       if (lane < K) {
-        sel_idx[warp * K + lane] = e;
-        sel_w[warp * K + lane] = wt;
-        atomicOr(&bitmap[e >> 5], 1u << (e & 31));
+        const int wq = e >> 5;
+        int r = __popc(bitmap[wq] & ((1u << (e & 31)) - 1u));
+        for (int w2 = 0; w2 < wq; ++w2) r += __popc(bitmap[w2]);
+        tokj[r * kMaxTok + warp] = (int8_t)lane;
+        tokw[r * kMaxTok + warp] = wt;
         if (blockIdx.x == 0 && a.idx_out) {
           a.idx_out[warp * K + lane] = e;
           a.w_out[warp * K + lane] = wt;
         }
       }
     }
-    named_bar(kBarConsumers, kConsumers);
-    if (warp == 0) {
+    if (warp == kConsumerWarps - 1) {
       const uint32_t word = bitmap[lane];
       const uint32_t cnt = __popc(word);
       uint32_t incl = cnt;
@@ -325,7 +326,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         if (lane >= off) incl += v;
       }
       const uint32_t pre = incl - cnt;
-      wpre[lane] = pre;
       uint32_t wbits = word;
       for (uint32_t r = pre; wbits; ++r) {
         const int b = __ffs(wbits) - 1;
@@ -333,13 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         ent[r] = lane * 32 + b;
       }
       const int U = __shfl_sync(0xffffffffu, (int)incl, 31);
-      __syncwarp();
-      for (int i = lane; i < T * K; i += 32) {
-        const int t = i / K, j = i % K, e = sel_idx[i];
-        const int r = wpre[e >> 5] + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
-        tokj[r * kMaxTok + t] = (int8_t)j;
-        tokw[r * kMaxTok + t] = sel_w[i];
-      }
       if (lane < T) {
         tokj[U * kMaxTok + lane] = (int8_t)K;  // shared expert: slot k, weight 1
         tokw[U * kMaxTok + lane] = 1.f;

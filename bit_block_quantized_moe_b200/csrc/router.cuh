@@ -118,7 +118,7 @@ __device__ __forceinline__ float load_logit(const float *row, int e) {
 }
 
 template <int NPL, bool kSmem = false>
-__device__ __forceinline__ void warp_topk_regs(const float *row, int E, int k, int lane, int &e_out, float &w_out) {
+__device__ __forceinline__ void warp_topk_regs_sel(const float *row, int E, int k, int lane, int &e_out, float &v_out) {
   float v[NPL];
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
@@ -153,7 +153,14 @@ __device__ __forceinline__ void warp_topk_regs(const float *row, int E, int k, i
     }
   }
   e_out = mye;
-  w_out = topk_softmax(myv, lane, k);
+  v_out = myv;
+}
+
+template <int NPL, bool kSmem = false>
+__device__ __forceinline__ void warp_topk_regs(const float *row, int E, int k, int lane, int &e_out, float &w_out) {
+  float v;
+  warp_topk_regs_sel<NPL, kSmem>(row, E, k, lane, e_out, v);
+  w_out = topk_softmax(v, lane, k);
 }
 
 // Top-k of one token's logits (one warp): k rounds, each taking the largest
@@ -213,8 +220,8 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // kFull: E == 32 * NPL, so every lane loads all its values with no bounds test
 // (the run-time test around each load costs about 1.7k cycles per call on B200).
 template <int NPL, bool kSmem = false, bool kFull = false>
-__device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, int lane, uint64_t *scratch,
-                                               int &e_out, float &w_out) {
+__device__ __forceinline__ void warp_topk_fast_sel(const float *row, int E, int k, int lane, uint64_t *scratch,
+                                                   int &e_out, float &v_out) {
   uint32_t kv[NPL];
   uint32_t mk = 0;
 #pragma unroll
@@ -240,7 +247,7 @@ __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, i
   const int total = __reduce_add_sync(0xffffffffu, cnt);
   if (total > 32) {
     __syncwarp();
-    warp_topk_regs<NPL, kSmem>(row, E, k, lane, e_out, w_out);
+    warp_topk_regs_sel<NPL, kSmem>(row, E, k, lane, e_out, v_out);
     return;
   }
   int pos = cnt;  // exclusive prefix of the candidate counts
@@ -268,7 +275,16 @@ __device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, i
   const uint64_t mine = lane < k ? scratch[32 + lane] : 0ull;
   __syncwarp();
   e_out = (int)~(uint32_t)mine;
-  w_out = topk_softmax(key_float((uint32_t)(mine >> 32)), lane, k);
+  v_out = key_float((uint32_t)(mine >> 32));
+}
+
+// Selection and weights (fp32 softmax over the k winners, lane j < k holding winner j).
+template <int NPL, bool kSmem = false, bool kFull = false>
+__device__ __forceinline__ void warp_topk_fast(const float *row, int E, int k, int lane, uint64_t *scratch,
+                                               int &e_out, float &w_out) {
+  float v;
+  warp_topk_fast_sel<NPL, kSmem, kFull>(row, E, k, lane, scratch, e_out, v);
+  w_out = topk_softmax(v, lane, k);
 }
 
 }  // namespace moe
