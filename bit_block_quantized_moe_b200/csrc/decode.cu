@@ -9,12 +9,15 @@
 //     -- grid barrier: all logits written.  Between arriving and waiting the
 //        CTA prepares its token rows as the MMA B operand (block correction
 //        sums, the (4c+2, 4c+3) pairs scaled by 1/4) --
-//  B  One warp per token reads its logits from L2, selects the top-k
-//     (threshold + rank) and marks its experts in a bit map (the tables were
-//     cleared while waiting on the barrier).  Then a spare warp builds the
-//     same sorted list of touched experts plus the shared expert as every
-//     other CTA, while the token warps compute their weights (softmax over
-//     their winners) and fill their table entries.
+//  B  One warp per token reads its logits from L2 and selects the top-k
+//     (threshold + rank); its weights are the softmax over its winners.
+//     Work entries: for T <= 3 one per (token, slot), fixed in advance, plus
+//     the shared expert (an expert two tokens chose is streamed twice; the
+//     weights are computed while phase D waits for h); for
+//     larger T the sorted list of touched experts plus the shared expert,
+//     built by a spare warp from a bit map of the winners while the token
+//     warps fill their table entries (the tables were cleared while waiting
+//     on the barrier).  Every CTA builds the same entries.
 //  C  Work lists, expert-major, cut into equal contiguous ranges per CTA:
 //     gate/up units (expert, 8 intermediate rows) and down stages (expert, two
 //     16-row units).  Stage s belongs to warp s % 14, which copies it into its
@@ -52,6 +55,7 @@ constexpr int kThreads = kConsumers;  // every warp computes and streams its own
 constexpr int kMaxTok = 8;
 constexpr int kMaxSel = 128;              // T * top_k
 constexpr int kMaxEntries = kMaxSel + 1;  // touched experts + shared
+constexpr int kSlotTokens = 3;            // up to this many tokens: one work entry per (token, slot)
 constexpr int kMaxE = 1024;
 constexpr int kMaxI = 512;                // down K handled by the h cache
 constexpr int kBarConsumers = 1;          // named barrier id (0 = __syncthreads)
@@ -80,7 +84,7 @@ struct DecodeArgs {
 };
 
 struct SmemLayout {
-  uint32_t xs, corr, hcorr, rpart, red, bitmap, ent, tokj, tokw, misc, ring, total;
+  uint32_t xs, corr, hcorr, rpart, red, bitmap, slv, ent, tokj, tokw, misc, ring, total;
 };
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -101,6 +105,8 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
   L.bitmap = o;
   o += (kMaxE / 32) * 4;
+  L.slv = o;  // slot entries: the winners' logits, token-major
+  o += kMaxSel * 4;
   L.ent = o;
   o = align_to(o + kMaxEntries * 4, 16);
   L.tokj = o;
@@ -200,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   float *rpart = reinterpret_cast<float *>(smem + L.rpart);
   float *red = reinterpret_cast<float *>(smem + L.red);
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + L.bitmap);
+  float *slv = reinterpret_cast<float *>(smem + L.slv);
   int *ent = reinterpret_cast<int *>(smem + L.ent);
   int8_t *tokj = reinterpret_cast<int8_t *>(smem + L.tokj);
   float *tokw = reinterpret_cast<float *>(smem + L.tokw);
@@ -299,47 +306,67 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         warp_topk_fast_sel<32, false>(row, E, K, lane, scratch, e, lv);
       if (lane < K) atomicOr(&bitmap[e >> 5], 1u << (e & 31));
     }
-    named_bar(kBarConsumers, kConsumers);  // every selected expert is in the bit map
-    if (warp < T) {
-      // While a spare warp builds the list: the token's weights (fp32 softmax over its winners) and its
-      // table entries, each lane ranking its expert among the touched ones from the bit map.
-      const float wt = topk_softmax(lv, lane, K);
-      if (lane < K) {
-        const int wq = e >> 5;
-        int r = __popc(bitmap[wq] & ((1u << (e & 31)) - 1u));
-        for (int w2 = 0; w2 < wq; ++w2) r += __popc(bitmap[w2]);
-        tokj[r * kMaxTok + warp] = (int8_t)lane;
-        tokw[r * kMaxTok + warp] = wt;
-        if (blockIdx.x == 0 && a.idx_out) {
-          a.idx_out[warp * K + lane] = e;
-          a.w_out[warp * K + lane] = wt;
+    if (T <= kSlotTokens && T * K <= E) {
+      // Slot entries: entry t * k + j is token t's j-th winner and the shared expert comes last, so the
+      // work split is fixed before the routing is known and no list is built; an expert that two tokens
+      // chose is streamed once per token.  The weights are computed later, while the CTA waits for h.
+      if (warp < T && lane < K) {
+        const int entry = warp * K + lane;
+        ent[entry] = e;
+        tokj[entry * kMaxTok + warp] = (int8_t)lane;
+        slv[entry] = lv;
+      }
+      if (warp == kConsumerWarps - 1 && lane < T) {
+        tokj[T * K * kMaxTok + lane] = (int8_t)K;  // shared expert: slot k, weight 1
+        tokw[T * K * kMaxTok + lane] = 1.f;
+        if (lane == 0) {
+          ent[T * K] = E;
+          misc[0] = T * K + 1;
         }
       }
-    }
-    if (warp == kConsumerWarps - 1) {
-      const uint32_t word = bitmap[lane];
-      const uint32_t cnt = __popc(word);
-      uint32_t incl = cnt;
+    } else {
+      named_bar(kBarConsumers, kConsumers);  // every selected expert is in the bit map
+      if (warp < T) {
+        // While a spare warp builds the list: the token's weights (fp32 softmax over its winners) and its
+        // table entries, each lane ranking its expert among the touched ones from the bit map.
+        const float wt = topk_softmax(lv, lane, K);
+        if (lane < K) {
+          const int wq = e >> 5;
+          int r = __popc(bitmap[wq] & ((1u << (e & 31)) - 1u));
+          for (int w2 = 0; w2 < wq; ++w2) r += __popc(bitmap[w2]);
+          tokj[r * kMaxTok + warp] = (int8_t)lane;
+          tokw[r * kMaxTok + warp] = wt;
+          if (blockIdx.x == 0 && a.idx_out) {
+            a.idx_out[warp * K + lane] = e;
+            a.w_out[warp * K + lane] = wt;
+          }
+        }
+      }
+      if (warp == kConsumerWarps - 1) {
+        const uint32_t word = bitmap[lane];
+        const uint32_t cnt = __popc(word);
+        uint32_t incl = cnt;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      const uint32_t pre = incl - cnt;
-      uint32_t wbits = word;
-      for (uint32_t r = pre; wbits; ++r) {
-        const int b = __ffs(wbits) - 1;
-        wbits &= wbits - 1;
-        ent[r] = lane * 32 + b;
-      }
-      const int U = __shfl_sync(0xffffffffu, (int)incl, 31);
-      if (lane < T) {
-        tokj[U * kMaxTok + lane] = (int8_t)K;  // shared expert: slot k, weight 1
-        tokw[U * kMaxTok + lane] = 1.f;
-      }
-      if (lane == 0) {
-        ent[U] = E;
-        misc[0] = U + 1;
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        const uint32_t pre = incl - cnt;
+        uint32_t wbits = word;
+        for (uint32_t r = pre; wbits; ++r) {
+          const int b = __ffs(wbits) - 1;
+          wbits &= wbits - 1;
+          ent[r] = lane * 32 + b;
+        }
+        const int U = __shfl_sync(0xffffffffu, (int)incl, 31);
+        if (lane < T) {
+          tokj[U * kMaxTok + lane] = (int8_t)K;  // shared expert: slot k, weight 1
+          tokw[U * kMaxTok + lane] = 1.f;
+        }
+        if (lane == 0) {
+          ent[U] = E;
+          misc[0] = U + 1;
+        }
       }
     }
   }
@@ -447,6 +474,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   const int hstride = I + 16;
   const int e_lo = d1 > d0 ? d0 / G.dn_units : 0;
   const int n_hc = d1 > d0 ? (d1 - 1) / G.dn_units - e_lo + 1 : 0;
+  if (T <= kSlotTokens && T * K <= E && warp < T) {
+    // slot entries: the token's weights, fp32 softmax over its winners (the down stages read them)
+    const float wt = topk_softmax(lane < K ? slv[warp * K + lane] : 0.f, lane, K);
+    if (lane < K) {
+      tokw[(warp * K + lane) * kMaxTok + warp] = wt;
+      if (blockIdx.x == 0 && a.idx_out) {
+        a.idx_out[warp * K + lane] = ent[warp * K + lane];
+        a.w_out[warp * K + lane] = wt;
+      }
+    }
+  }
   if (tid < n_hc && !*reinterpret_cast<volatile int *>(&misc[1])) {
     const uint64_t t0 = global_timer_ns();
     while (ld_acquire_gpu(&ready[e_lo + tid]) < (uint32_t)G.gu_units) {
