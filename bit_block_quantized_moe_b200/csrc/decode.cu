@@ -374,10 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
 
   const int nent = misc[0];
   const int n_gu = nent * G.gu_units, n_dn = nent * G.dn_units;
-  const int g0 = (int)((long long)n_gu * blockIdx.x / gridDim.x);
-  const int g1 = (int)((long long)n_gu * (blockIdx.x + 1) / gridDim.x);
-  const int d0 = (int)((long long)n_dn * blockIdx.x / gridDim.x);
-  const int d1 = (int)((long long)n_dn * (blockIdx.x + 1) / gridDim.x);
+  // contiguous shares of the units (32-bit products: at most 129 entries x 256 units x the grid)
+  const int g0 = (int)((uint32_t)n_gu * blockIdx.x / gridDim.x);
+  const int g1 = (int)((uint32_t)n_gu * (blockIdx.x + 1) / gridDim.x);
+  const int d0 = (int)((uint32_t)n_dn * blockIdx.x / gridDim.x);
+  const int d1 = (int)((uint32_t)n_dn * (blockIdx.x + 1) / gridDim.x);
   const int pps = 2;  // down units (16 rows) per stage: enough stages to keep every warp busy
   const int n_gu_st = g1 - g0;
   const int n_dn_st = (d1 - d0 + pps - 1) / pps;
@@ -461,10 +462,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   // Publish this CTA's finished gate/up units per expert (one fence for all of them).
   named_bar(kBarConsumers, kConsumers);
   if (tid == 0 && g1 > g0) {
-    __threadfence();
+    // release: the CTA's h stores (ordered before by the barrier) before the counts; no value returned
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
     for (int entry = g0 / G.gu_units; entry <= (g1 - 1) / G.gu_units; ++entry) {
       const int lo = max(g0, entry * G.gu_units), hi = min(g1, (entry + 1) * G.gu_units);
-      atomicAdd(&ready[entry], (uint32_t)(hi - lo));
+      asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(&ready[entry]), "r"((uint32_t)(hi - lo)) : "memory");
     }
   }
 

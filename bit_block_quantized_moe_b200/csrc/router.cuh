@@ -13,7 +13,8 @@ namespace moe {
 // identical routing decisions.  kT is the token count when it is fixed at
 // compile time (0: T at run time); the arithmetic is the same either way, but a
 // run-time T leaves all 8 token slots in the code behind predicates, about
-// twice the cycles for T = 3 on B200 (router_part_any picks the instance).
+// twice the cycles for T = 3 on B200 (router_part_any picks the instance: compile-time
+// T for the decode window T <= 3, the 8-slot code for larger windows).
 constexpr int kRouterParts = 2;
 template <bool kWrShared, int kT = 0>
 __device__ __forceinline__ void router_part(const uint16_t *x, int xstride, int T_, const float *wrow, int H,
@@ -56,11 +57,7 @@ __device__ __forceinline__ void router_part_any(const uint16_t *x, int xstride, 
     case 1: router_part<kWrShared, 1>(x, xstride, T, wrow, H, part, lane, acc); break;
     case 2: router_part<kWrShared, 2>(x, xstride, T, wrow, H, part, lane, acc); break;
     case 3: router_part<kWrShared, 3>(x, xstride, T, wrow, H, part, lane, acc); break;
-    case 4: router_part<kWrShared, 4>(x, xstride, T, wrow, H, part, lane, acc); break;
-    case 5: router_part<kWrShared, 5>(x, xstride, T, wrow, H, part, lane, acc); break;
-    case 6: router_part<kWrShared, 6>(x, xstride, T, wrow, H, part, lane, acc); break;
-    case 7: router_part<kWrShared, 7>(x, xstride, T, wrow, H, part, lane, acc); break;
-    default: router_part<kWrShared, 8>(x, xstride, T, wrow, H, part, lane, acc); break;
+    default: router_part<kWrShared, 0>(x, xstride, T, wrow, H, part, lane, acc); break;
   }
 }
 
