@@ -224,6 +224,21 @@ def test_experts_forward_bad_index_sets_status(tiny):
     L.check_status()  # cleared
 
 
+@pytest.mark.parametrize("T", [2, 3, 4])
+def test_fused_decode_repeated_experts(full, T):
+    """Identical tokens choose the same experts, so every expert is chosen by all T tokens: T <= 3 streams it
+    once per (token, slot) entry, T = 4 once per touched expert.  Against the oracle, and the output rows are
+    equal bit for bit (each token's contributions are summed in the same order)."""
+    L, w = full
+    x1 = make_x(1, 2048, seed=55)
+    x = np.repeat(x1, T, axis=0)
+    y, idx, wts = gpu_forward(L, x)
+    assert all(np.array_equal(idx[t], idx[0]) and np.array_equal(wts[t], wts[0]) for t in range(T))
+    assert all(np.array_equal(y[t], y[0]) for t in range(T))
+    err, l2, flagged = check_layer(CONFIGS["prefill"], w, x, y, idx, wts)
+    print(f"repeated experts T={T}: max-rel {err:.3e} relL2 {l2:.3e}")
+
+
 @pytest.mark.parametrize("T", [4, 5, 8])
 def test_fused_decode_window_sizes(full, T):
     L, w = full
