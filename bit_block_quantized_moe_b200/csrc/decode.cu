@@ -222,15 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   float *wr_s = reinterpret_cast<float *>(ring);  // router rows live in the ring until phase C
 
   // ---------------- phase A: set-up, router ----------------
+  // The next launch on this stream may start its own set-up on the SMs this grid frees: it reads nothing
+  // that this grid writes before its griddepcontrol.wait.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0)
     for (int i = 0; i < 16; ++i) misc[i] = 0;
-  // The tokens, then this CTA's router rows: cp.async pieces from every thread
-  // (two commit groups), and an L2 prefetch of this CTA's slice of the shared expert.
-  for (int i = tid; i < T * (H / 8); i += kConsumers) {
-    const int t = i / (H / 8), c8 = i % (H / 8);
-    cp_async16(xs + t * xstride + c8 * 8, a.x + (size_t)t * H + c8 * 8);
-  }
-  cp_async_commit();
+  // This CTA's router rows (weights: no earlier launch writes them), cp.async pieces from every thread, and
+  // an L2 prefetch of this CTA's slice of the shared expert.
   for (int i = tid; i < n_rrows * (H / 4); i += kConsumers) {
     const int r = i / (H / 4), c4 = i % (H / 4);
     cp_async16(wr_s + (size_t)r * H + c4 * 4, a.Wr + (size_t)(blockIdx.x + (size_t)gridDim.x * r) * H + c4 * 4);
@@ -244,6 +242,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       for (size_t o = 0; o < n; o += 32768) bulk_prefetch_l2(a.shared + off + o, (uint32_t)min((size_t)32768, n - o));
     }
   }
+  // Everything below may depend on the previous launch on this stream (its outputs, the workspace).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  uint64_t bar_target = 0;  // the grid barrier's leader (the last thread) reads the launch counter now
+  if (tid == kConsumers - 1) {
+    const uint64_t c0 = *reinterpret_cast<volatile uint64_t *>(a.gbar);
+    bar_target = (c0 / gridDim.x + 1) * gridDim.x;
+  }
+  for (int i = tid; i < T * (H / 8); i += kConsumers) {
+    const int t = i / (H / 8), c8 = i % (H / 8);
+    cp_async16(xs + t * xstride + c8 * 8, a.x + (size_t)t * H + c8 * 8);
+  }
+  cp_async_commit();
   for (int i = tid; i < xstride / 8; i += kConsumers)
     reinterpret_cast<uint4 *>(xs + T * xstride)[i] = make_uint4(0u, 0u, 0u, 0u);
   {
@@ -281,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     // The barrier's leader is the last thread, which has the fewest token-row pieces to prepare, so
     // that its fence and atomic round trip overlap the others' preparation.
     const bool leader = tid == kConsumers - 1;
-    const uint64_t bar_target = grid_arrive(a.gbar, kBarConsumers, kConsumers, leader);
+    grid_arrive_release(a.gbar, kBarConsumers, kConsumers, leader);
     prep_rows(xs, xstride, H, T, corr, tid);
     // the touched-expert tables start empty (filled once the top-k is known)
     for (int i = tid; i < kMaxEntries * kMaxTok; i += kConsumers) {
@@ -699,11 +709,13 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   trace_mark(MOE_KERNEL_DECODE_FUSED, false, s);
   err = cudaLaunchKernelEx(&cfg, kern, a);
   trace_mark(MOE_KERNEL_DECODE_FUSED, true, s);

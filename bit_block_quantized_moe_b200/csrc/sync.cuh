@@ -133,24 +133,22 @@ __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
   return v;
 }
 
-// Grid-wide barrier for a co-resident (cooperatively launched) grid, over one
-// monotonic 64-bit arrival counter (zeroed once with the workspace, never
-// reset), split in two so that independent work can run between arriving and
-// waiting.  grid_arrive: the participating threads of each CTA meet at named
-// barrier `bar_id`; thread `leader` fences, adds 1 and returns the count the
-// wait must reach (the next multiple of gridDim.x).  grid_wait: the leader
-// polls until the counter reaches it, then the threads meet again.  One atomic
-// round trip per CTA.  grid_wait returns false (and sets the status timeout
-// bit) if the wait hit the limit.
-__device__ __forceinline__ uint64_t grid_arrive(uint64_t *count, int bar_id, int nthreads, bool leader) {
+// Grid barrier of a cooperatively launched (all CTAs resident) grid over one
+// monotonic 64-bit launch counter (zeroed once with the workspace, never
+// reset: every CTA adds 1 per launch), split in two so that independent work
+// can run between arriving and waiting.  The leader reads the counter at
+// kernel start and derives the target; grid_arrive_release: the participating
+// threads meet at named barrier `bar_id`, the leader's release add publishes
+// the CTA's earlier writes.  grid_wait: the leader polls (acquire) until the
+// counter reaches the target, then the threads meet again; it returns false
+// (and sets the status timeout bit) if the wait hit the limit.
+
+// Arrival with the target known in advance: the leader read the counter at kernel start (before any CTA of
+// this launch can have added all of its arrivals, it holds launch * grid plus fewer than grid), so the target
+// is the next multiple of the grid size; the arrival is a release add whose value nobody waits for.
+__device__ __forceinline__ void grid_arrive_release(uint64_t *count, int bar_id, int nthreads, bool leader) {
   named_bar(bar_id, nthreads);
-  uint64_t target = 0;
-  if (leader) {
-    __threadfence();
-    const unsigned long long old = atomicAdd(reinterpret_cast<unsigned long long *>(count), 1ull);
-    target = (old / gridDim.x + 1) * gridDim.x;
-  }
-  return target;
+  if (leader) asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(count) : "memory");
 }
 
 __device__ __forceinline__ bool grid_wait(const uint64_t *count, uint64_t target, int bar_id, int nthreads,

@@ -58,7 +58,12 @@ typedef struct CUstream_st *moe_stream_t;
  * n_experts <= 1024 takes one fused persistent kernel for the whole layer;
  * other T <= 8 shapes take the routing kernels plus register-dequantising
  * tensor-core expert kernels (slower, about 2x at the pages' shape); T > 8
- * takes the tcgen05 prefill kernels. */
+ * takes the tcgen05 prefill kernels.  The fused kernel is launched with
+ * programmatic dependent launch: while an earlier fused launch on the same
+ * stream finishes, it may already load its router rows and prefetch the
+ * shared expert (weights, which no launch of this library writes); it reads
+ * x and the workspace only after that launch has completed, and every other
+ * earlier work on the stream completes before it starts. */
 typedef struct {
   int32_t hidden;    /* H: model width (router and expert input/output size) */
   int32_t inter;     /* I: expert intermediate size (gate/up rows, down columns) */
@@ -121,7 +126,7 @@ moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_ex
  * Host.  Bytes of scratch memory moe_route / moe_layer_forward /
  * moe_experts_forward need for up to max_T tokens (0 if invalid).  Its first
  * 256 bytes hold the sticky device status word (offset 0) and the decode
- * kernel's grid-barrier counter (offset 64): zero the workspace (or at least
+ * kernel's launch counter (offset 64, its grid barrier): zero the workspace (or at least
  * those 256 bytes) once after allocating it, and again after a call reported
  * MOE_ERR_TIMEOUT.  One workspace must not be used by two calls that can run
  * at the same time.  A workspace of moe_workspace_bytes(dims, max_T) serves
