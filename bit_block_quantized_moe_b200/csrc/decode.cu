@@ -2,10 +2,12 @@
 // cooperatively launched kernel (sm_100a).  One CTA per SM, 14 warps, each of
 // which both streams and computes.
 //
-//  A  Every thread copies (cp.async, 16 B) its pieces of the tokens and of this
-//     CTA's router rows into shared memory; one thread prefetches the CTA's
-//     slice of the shared expert into L2.  2 warps per router row (one half of
-//     K each) write the logits.
+//  A  Every thread copies (cp.async, 16 B) its pieces of this CTA's router
+//     rows into shared memory and one thread prefetches the CTA's slice of the
+//     shared expert into L2; launched as a programmatic dependent of the
+//     previous decode launch, the CTA does this while that launch finishes and
+//     only then (griddepcontrol.wait) copies the tokens.  2 warps per router
+//     row (one half of K each) write the logits.
 //     -- grid barrier: all logits written.  Between arriving and waiting the
 //        CTA prepares its token rows as the MMA B operand (block correction
 //        sums, the (4c+2, 4c+3) pairs scaled by 1/4) --
@@ -29,8 +31,8 @@
 //  D  Once the h of the (at most two) experts in the CTA's down range is
 //     complete (per-expert counter, bounded wait) it is copied into shared
 //     memory; each down stage (two 16-row units) again belongs to one warp:
-//     partial = w[t, e] * (Wd_e h_e) per (expert, tile).  The warp that writes
-//     a tile's last partial sums them in expert order and writes out (bf16).
+//     partial = w[t, e] * (Wd_e h_e) per (entry, tile).  The warp that writes
+//     a tile's last partial sums them in entry order and writes out (bf16).
 // Dequantisation happens in registers: the 2-bit codes of a row OR into the
 // mantissa of bf16 128.0 (128 + q, or 128 + 4q with the matching activation
 // pair pre-scaled by 1/4), one logic op per pair of weights, and feed
@@ -287,9 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       named_bar(kBarConsumers, kConsumers);
     }
     // Arrive on the grid barrier, prepare the token rows as the B operand while the other CTAs finish
-    // their logits (the router is done with them), then wait.
-    // The barrier's leader is the last thread, which has the fewest token-row pieces to prepare, so
-    // that its fence and atomic round trip overlap the others' preparation.
+    // their logits (the router is done with them), then wait.  The barrier's leader (the last thread,
+    // which has the fewest token-row pieces to prepare) read the launch counter at the start.
     const bool leader = tid == kConsumers - 1;
     grid_arrive_release(a.gbar, kBarConsumers, kConsumers, leader);
     prep_rows(xs, xstride, H, T, corr, tid);
@@ -656,9 +657,9 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   const int ns = nw;
   const SmemLayout L = smem_layout(T, G.H, ns, stage_bytes);
   if (L.total > (uint32_t)max_smem) return cudaErrorInvalidConfiguration;
-  // the per-CTA down range must fit the 128-entry completed-tile list
+  // a CTA's down range spans at most two entries (the h cache of phase D holds two): at most dn_units units
   const int max_entries = min(T * d.top_k, d.n_experts) + 1;
-  if ((max_entries * G.dn_units + n_sm - 1) / n_sm > kMaxSel) return cudaErrorInvalidConfiguration;
+  if ((max_entries * G.dn_units + n_sm - 1) / n_sm > G.dn_units) return cudaErrorInvalidConfiguration;
   const int rrows = (d.n_experts + n_sm - 1) / n_sm;  // router rows per CTA, staged in the ring
   if ((size_t)rrows * d.hidden * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;
   if ((size_t)T * d.n_experts * 4 > (size_t)ns * stage_bytes) return cudaErrorInvalidConfiguration;  // logits
