@@ -521,16 +521,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   for (int he = 0; he < n_hc; ++he) prep_rows(hc + he * T * hstride, hstride, I, T, hcorr + he * (kMaxI / 32) * kMaxTok, tid);
   named_bar(kBarConsumers, kConsumers);
 
-  // Sums a finished output tile's partials in expert order (deterministic) and writes its rows.
+  // Sums a finished output tile's partials in a fixed order (deterministic) and writes its rows.
+  // A lane's column c holds tokens 2c, 2c + 1, so only ceil(T / 2) columns carry tokens: the
+  // lanes of the other columns take a share of the entries instead.  cu columns (a power of
+  // two) are summed, each by 4 / cu lanes over the entries e = sub (mod 4 / cu) in order, and
+  // the lanes' sums are added in a fixed butterfly (every lane ends with the same bits).
   auto reduce_tile = [&](int tile) {
+    const int cu = T <= 2 ? 1 : (T <= 4 ? 2 : 4), nsub = 4 / cu, sub = c / cu, cc = c % cu;
     float o[4] = {0.f, 0.f, 0.f, 0.f};
-    const float *pp = a.partial + (size_t)tile * 128 + lane * 4;
-    int e2 = 0;
-    for (; e2 < nent; e2 += 16) {  // up to sixteen loads in flight, summed in expert order
+    const float *pp = a.partial + (size_t)tile * 128 + (4 * g + cc) * 4;
+    const size_t est = (size_t)G.dn_units * 128;
+    for (int e2 = sub; e2 < nent; e2 += 16 * nsub) {  // up to sixteen loads in flight per lane
       float4 v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u)
-        v[u] = e2 + u < nent ? ldg_cg_f4(pp + (size_t)(e2 + u) * G.dn_units * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = e2 + u * nsub < nent ? ldg_cg_f4(pp + (size_t)(e2 + u * nsub) * est) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         o[0] += v[u].x;
@@ -539,18 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         o[3] += v[u].w;
       }
     }
-    for (; e2 < nent; ++e2) {
-      const float4 v = ldg_cg_f4(pp + (size_t)e2 * G.dn_units * 128);
-      o[0] += v.x;
-      o[1] += v.y;
-      o[2] += v.z;
-      o[3] += v.w;
-    }
+    for (int m = cu; m < 4; m <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], m);
     const int r0 = 16 * tile + g;
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int n = 2 * c + hf;
-      if (n < T) {
+      if (sub == 0 && n < T) {
         if (a.out_f32) {
           a.out_f32[(size_t)n * H + r0] = o[hf];
           a.out_f32[(size_t)n * H + r0 + 8] = o[2 + hf];
@@ -587,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
       *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
       // Count the contribution; the warp that brings the tile's last one sums all its
-      // partials in expert order right away and writes the output rows.  The warp sync orders
+      // partials in a fixed order right away and writes the output rows.  The warp sync orders
       // every lane's partial store before lane 0's release; the count is one acquire-release
       // atomic at GPU scope, so the last contributor also acquires every other partial (a full
       // fence on both sides cost 0.3-0.5 us more per step).
