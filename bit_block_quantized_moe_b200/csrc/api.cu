@@ -60,7 +60,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_h = take(slots * I * 2);
   const size_t o_y = take(slots * H * 4);
   const bool fused = decode_fused_supported(d, T);
-  const size_t o_tcnt = take(fused ? decode_counter_words(d) * 4 : 0);
+  const size_t o_ready = take(fused ? decode_counter_words(d) * 4 : 0);
   const size_t o_part = take(fused ? decode_partial_floats(d, T) * 4 : 0);
   const bool rtc = router_tc_supported(d, T);
   const size_t o_wsplit = take(rtc ? (size_t)3 * E * H * 2 : 0);
@@ -92,7 +92,7 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->h = reinterpret_cast<uint16_t *>(b + o_h);
     ws->y = reinterpret_cast<float *>(b + o_y);
     ws->gbar = reinterpret_cast<uint64_t *>(b + o_hdr + 64);
-    ws->tile_cnt = reinterpret_cast<uint32_t *>(b + o_tcnt);
+    ws->ready = reinterpret_cast<uint32_t *>(b + o_ready);
     ws->partial = reinterpret_cast<float *>(b + o_part);
     ws->wsplit = rtc ? reinterpret_cast<uint16_t *>(b + o_wsplit) : nullptr;
     ws->rpart = reinterpret_cast<float *>(b + o_rpart);

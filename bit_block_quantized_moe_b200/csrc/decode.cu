@@ -31,8 +31,10 @@
 //  D  Once the h of the (at most two) experts in the CTA's down range is
 //     complete (per-expert counter, bounded wait) it is copied into shared
 //     memory; each down stage (two 16-row units) again belongs to one warp:
-//     partial = w[t, e] * (Wd_e h_e) per (entry, tile).  The warp that writes
-//     a tile's last partial sums them in entry order and writes out (bf16).
+//     partial = w[t, e] * (Wd_e h_e) per (entry, tile).
+//     -- second grid barrier: all partials written --
+//     One warp per output tile sums its partials in a fixed order and writes
+//     out (bf16, or fp32).
 // Dequantisation happens in registers: the 2-bit codes of a row OR into the
 // mantissa of bf16 128.0 (128 + q, or 128 + 4q with the matching activation
 // pair pre-scaled by 1/4), one logic op per pair of weights, and feed
@@ -73,7 +75,7 @@ struct DecodeArgs {
   float *logits;       // [T][E]
   uint16_t *h;         // [T][k+1][I]
   float *partial;      // [entries][dn_units][32][4]
-  uint32_t *tile_cnt;  // [dn_units] then ready[kMaxEntries]
+  uint32_t *ready;     // [kMaxEntries] per-entry count of finished gate/up units
   uint64_t *gbar;      // monotonic grid-barrier arrival counter
   int32_t *idx_out;    // optional [T][k]
   float *w_out;        // optional [T][k]
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   float *tokw = reinterpret_cast<float *>(smem + L.tokw);
   int *misc = reinterpret_cast<int *>(smem + L.misc);
   uint8_t *ring = smem + L.ring;
-  uint32_t *ready = a.tile_cnt + G.dn_units;
+  uint32_t *ready = a.ready;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   }
   // Everything below may depend on the previous launch on this stream (its outputs, the workspace).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  uint64_t bar_target = 0;  // the grid barrier's leader (the last thread) reads the launch counter now
+  uint64_t bar_target = 0;  // the grid barriers' leader (the last thread) reads the arrival counter now
   if (tid == kConsumers - 1) {
     const uint64_t c0 = *reinterpret_cast<volatile uint64_t *>(a.gbar);
     bar_target = (c0 / gridDim.x + 1) * gridDim.x;
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     reinterpret_cast<uint4 *>(xs + T * xstride)[i] = make_uint4(0u, 0u, 0u, 0u);
   {
     if (blockIdx.x == 0)
-      for (int i = tid; i < G.dn_units + kMaxEntries; i += kConsumers) a.tile_cnt[i] = 0u;
+      for (int i = tid; i < kMaxEntries; i += kConsumers) ready[i] = 0u;
     constexpr int kRowsPerPass = kConsumerWarps / kRouterParts;  // one warp per router row part
     // the bias of the logit this thread finishes in the first pass, loaded while the copies land
     float bias0 = 0.f;
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
     }
     // Arrive on the grid barrier, prepare the token rows as the B operand while the other CTAs finish
     // their logits (the router is done with them), then wait.  The barrier's leader (the last thread,
-    // which has the fewest token-row pieces to prepare) read the launch counter at the start.
+    // which has the fewest token-row pieces to prepare) read the arrival counter at the start.
     const bool leader = tid == kConsumers - 1;
     grid_arrive_release(a.gbar, kBarConsumers, kConsumers, leader);
     prep_rows(xs, xstride, H, T, corr, tid);
@@ -587,21 +589,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       const float o4[4] = {acc[0] * w0, acc[1] * w1, acc[2] * w0, acc[3] * w1};
       float *pp = a.partial + ((size_t)entry * G.dn_units + tile) * 128;
       *reinterpret_cast<float4 *>(pp + lane * 4) = make_float4(o4[0], o4[1], o4[2], o4[3]);
-      // Count the contribution; the warp that brings the tile's last one sums all its
-      // partials in a fixed order right away and writes the output rows.  The warp sync orders
-      // every lane's partial store before lane 0's release; the count is one acquire-release
-      // atomic at GPU scope, so the last contributor also acquires every other partial (a full
-      // fence on both sides cost 0.3-0.5 us more per step).
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = atom_add_acq_rel_gpu(&a.tile_cnt[tile], 1u) == (uint32_t)(nent - 1);
-      if (__shfl_sync(0xffffffffu, last, 0)) {
-        __syncwarp();
-        reduce_tile(tile);
-      }
     }
   }
 
+  // Second grid barrier: once every CTA has passed it, every partial of this launch is written
+  // (the arrival's release add publishes the CTA's partial stores).  Then the output tiles are
+  // shared out, the CTA's k-th tile to warp k mod 14.  One arrival per CTA replaces a counted,
+  // acquire-release atomic per unit (two per warp, about 1 us each on the warp's path).
+  {
+    const bool leader = tid == kConsumers - 1;
+    grid_arrive_release(a.gbar, kBarConsumers, kConsumers, leader);
+    if (grid_wait(a.gbar, bar_target + gridDim.x, kBarConsumers, kConsumers, leader, a.status, &misc[2]))
+      for (int k = 0, tile = blockIdx.x; tile < G.dn_units; ++k, tile += gridDim.x)
+        if (warp == k % kConsumerWarps) reduce_tile(tile);
+  }
   cp_async_wait_all();  // nothing of this thread's may still be landing when the CTA ends
 }
 
@@ -631,7 +632,7 @@ size_t decode_partial_floats(const moe_dims &d, int T) {
   return (size_t)entries * G.dn_units * 128;
 }
 
-size_t decode_counter_words(const moe_dims &d) { return (size_t)d.hidden / 16 + kMaxEntries; }
+size_t decode_counter_words(const moe_dims &) { return kMaxEntries; }
 
 cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const float *Wr, const float *bias,
                                 const uint8_t *experts, const uint8_t *shared, int T, const Workspace &ws,
@@ -678,7 +679,7 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   a.logits = ws.logits;
   a.h = ws.h;
   a.partial = ws.partial;
-  a.tile_cnt = ws.tile_cnt;
+  a.ready = ws.ready;
   a.gbar = ws.gbar;
   a.idx_out = idx_out;
   a.w_out = w_out;

@@ -29,7 +29,7 @@ struct Workspace {
   uint16_t *h;             // [T*k + T][I] bf16 SwiGLU outputs by sorted position
   float *y;                // [T*k + T][H] fp32 expert outputs by sorted position
   uint64_t *gbar;          // grid barrier of the fused decode kernel: monotonic arrival counter
-  uint32_t *tile_cnt;      // fused decode: per-tile arrival counters, then per-expert ready counters
+  uint32_t *ready;         // fused decode: per-entry ready counters (finished gate/up units)
   float *partial;          // fused decode: per (expert, tile) partial outputs
   uint16_t *wsplit;        // tcgen05 router: [3][E][H] bf16 planes of the router weights (null: legacy router)
   float *rpart;            // tcgen05 router: [ksplit][T][E] K-split partial logits (ksplit > 1)

@@ -112,17 +112,6 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   return v;
 }
 
-// Atomic add with acquire-release semantics at GPU scope; returns the old value.
-__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // Loads through L2 only (data written earlier in the same kernel by other CTAs).
 __device__ __forceinline__ uint2 ldg_cg_v2(const void *p) { return __ldcg(reinterpret_cast<const uint2 *>(p)); }
 __device__ __forceinline__ float4 ldg_cg_f4(const void *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
@@ -133,19 +122,21 @@ __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
   return v;
 }
 
-// Grid barrier of a cooperatively launched (all CTAs resident) grid over one
-// monotonic 64-bit launch counter (zeroed once with the workspace, never
-// reset: every CTA adds 1 per launch), split in two so that independent work
-// can run between arriving and waiting.  The leader reads the counter at
-// kernel start and derives the target; grid_arrive_release: the participating
-// threads meet at named barrier `bar_id`, the leader's release add publishes
-// the CTA's earlier writes.  grid_wait: the leader polls (acquire) until the
-// counter reaches the target, then the threads meet again; it returns false
-// (and sets the status timeout bit) if the wait hit the limit.
+// Grid barriers of a cooperatively launched (all CTAs resident) grid over one
+// monotonic 64-bit arrival counter (zeroed once with the workspace, never
+// reset: every CTA adds 1 per barrier, and every launch passes the same number
+// of barriers), each split in two so that independent work can run between
+// arriving and waiting.  The leader reads the counter at kernel start and
+// derives the targets; grid_arrive_release: the participating threads meet at
+// named barrier `bar_id`, the leader's release add publishes the CTA's earlier
+// writes.  grid_wait: the leader polls (acquire) until the counter reaches the
+// target, then the threads meet again; it returns false (and sets the status
+// timeout bit) if the wait hit the limit.
 
-// Arrival with the target known in advance: the leader read the counter at kernel start (before any CTA of
-// this launch can have added all of its arrivals, it holds launch * grid plus fewer than grid), so the target
-// is the next multiple of the grid size; the arrival is a release add whose value nobody waits for.
+// Arrival with the target known in advance: the leader read the counter at kernel start, before this CTA
+// arrived anywhere, so it held (earlier launches x barriers per launch) x grid plus fewer than grid; the
+// first barrier's target is the next multiple of the grid size, the i-th one i - 1 grid sizes beyond it.
+// The arrival is a release add whose value nobody waits for.
 __device__ __forceinline__ void grid_arrive_release(uint64_t *count, int bar_id, int nthreads, bool leader) {
   named_bar(bar_id, nthreads);
   if (leader) asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(count) : "memory");

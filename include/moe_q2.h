@@ -126,8 +126,8 @@ moe_status moe_pack_q2(const moe_dims *dims, const void *canonical, int32_t n_ex
  * Host.  Bytes of scratch memory moe_route / moe_layer_forward /
  * moe_experts_forward need for up to max_T tokens (0 if invalid).  Its first
  * 256 bytes hold the sticky device status word (offset 0) and the decode
- * kernel's launch counter (offset 64, its grid barrier): zero the workspace (or at least
- * those 256 bytes) once after allocating it, and again after a call reported
+ * kernel's grid-barrier arrival counter (offset 64): zero the workspace (or at
+ * least those 256 bytes) once after allocating it, and again after a call reported
  * MOE_ERR_TIMEOUT.  One workspace must not be used by two calls that can run
  * at the same time.  A workspace of moe_workspace_bytes(dims, max_T) serves
  * every T <= max_T.  For T > 8 it also holds the router weights split into
