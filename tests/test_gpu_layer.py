@@ -239,6 +239,30 @@ def test_fused_decode_repeated_experts(full, T):
     print(f"repeated experts T={T}: max-rel {err:.3e} relL2 {l2:.3e}")
 
 
+def test_fused_decode_barrier_counter(full):
+    """The fused kernel's two grid barriers each add one arrival per CTA to the workspace's monotonic counter
+    (offset 64), so every launch moves it by exactly twice the grid size (one CTA per SM) whatever T, and the
+    barrier targets a launch derives from the value it reads at start stay right across a run of mixed window
+    sizes on one workspace."""
+    L, w = full
+    L.reserve(8)
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+
+    def counter():
+        torch.cuda.synchronize()
+        return int(L.workspace[64:72].cpu().numpy().view(np.uint64)[0])
+
+    c = counter()
+    assert c % n_sm == 0
+    for i, T in enumerate((3, 1, 8, 2, 5, 3)):
+        x = make_x(T, 2048, seed=900 + i)
+        y, idx, wts = gpu_forward(L, x)
+        c2 = counter()
+        assert c2 - c == 2 * n_sm, (T, c, c2)
+        c = c2
+        check_layer(CONFIGS["prefill"], w, x, y, idx, wts)
+
+
 @pytest.mark.parametrize("T", [4, 5, 8])
 def test_fused_decode_window_sizes(full, T):
     L, w = full
