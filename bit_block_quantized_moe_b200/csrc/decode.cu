@@ -117,7 +117,7 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   o = align_to(o + kMaxEntries * kMaxTok, 16);
   L.tokw = o;
   o = align_to(o + kMaxEntries * kMaxTok * 4, 16);
-  L.misc = o;  // [0] entries [1] abort [2] barrier flag [3] done tiles
+  L.misc = o;  // [0] entries [1] abort [2] grid-barrier flag
   o += 64;
   L.ring = align_to(o, 128);
   L.total = L.ring + (uint32_t)ns * stage_bytes;

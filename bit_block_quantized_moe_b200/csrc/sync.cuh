@@ -60,25 +60,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   return true;
 }
 
-// ---- bulk copies (TMA engine, no tensor map) ---------------------------------------
-// global -> shared, completion counted in bytes on `bar`.  16-byte aligned, size % 16 == 0.
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 // ---- cp.async (load/store-unit path, 16 B per thread) ----------------------------
 // Many threads each moving 16-byte pieces keep far more bytes in flight per SM
 // than one thread issuing large bulk copies.
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
-}
-// One arrival on `bar` once every cp.async this thread issued so far has landed
-// (the barrier's expected count includes it).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -113,7 +99,6 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 }
 
 // Loads through L2 only (data written earlier in the same kernel by other CTAs).
-__device__ __forceinline__ uint2 ldg_cg_v2(const void *p) { return __ldcg(reinterpret_cast<const uint2 *>(p)); }
 __device__ __forceinline__ float4 ldg_cg_f4(const void *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
 
 __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
