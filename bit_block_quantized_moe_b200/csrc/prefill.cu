@@ -11,13 +11,14 @@
 //                      zeros) and two of the expert's token rows (slot-sorted
 //                      activations, 128-byte swizzle, 16/32/64/128-row boxes)
 //                      into one of 8 (5) shared-memory stages;
-//   16 dequant warps : decode the codes in registers to bf16 d * (q - 1)
-//                      while the tensor core still reads the A stage they
-//                      will fill, then store them (tcgen05.st), one 16-row
-//                      unit (4 blocks) per warp (half a unit with one M
-//                      tile); once the MMAs of a chunk
-//                      have completed they also release its shared-memory
-//                      stage to the producer;
+//   16 dequant warps : two groups of 8 on alternate chunks (one group's
+//                      waits and stores overlap the other's decode); each
+//                      warp decodes one 16-row unit (4 blocks) of every M
+//                      tile in registers to bf16 d * (q - 1) while the tensor
+//                      core still reads the A stage it will fill, then stores
+//                      them (tcgen05.st); once the MMAs of the group's
+//                      previous chunk have completed it also releases that
+//                      chunk's shared-memory stage to the producer;
 //   MMA warp        : 8 tcgen05.mma per M tile and chunk (A from tensor memory, B
 //                     from shared memory), fp32 accumulators in tensor
 //                     memory, one commit per chunk.  It waits only on the A
@@ -63,10 +64,9 @@ struct TcCfg {
   static constexpr int kAStages = 2;                              // tensor-memory A stages (MT x 64 columns)
   static constexpr uint32_t kDCols = MT * MAXN;                   // one accumulator buffer
   static constexpr uint32_t kTmemA0 = 2 * kDCols;                 // D buffers at 0 and kDCols, A stages after
-  static constexpr int kBlocksPerWarp = MT == 2 ? 4 : 2;          // blocks of its unit each dequant warp decodes
   static_assert(kTmemA0 + kAStages * MT * 64 <= kTmemCols, "tensor memory columns");
   static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment for the 128-byte swizzle");
-  static_assert(kNumDequant * kBlocksPerWarp == MT * kTileUnits * 4, "every block of a chunk decoded once");
+  static_assert(kAStages == 2 && kNumDequant == 16, "two dequant groups of 8, one per A stage");
 };
 using CfgFew = TcCfg<2, 64>;
 using CfgMany = TcCfg<1, 128>;
@@ -145,10 +145,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&B.full[i], 1);
-      mbar_init(&B.empty[i], kNumDequant);  // each dequant warp, once the stage's MMAs have completed
+      mbar_init(&B.empty[i], kNumDequant / 2);  // each warp of the group that read it, once its MMAs completed
     }
     for (int i = 0; i < kAStages; ++i) {
-      mbar_init(&B.afull[i], kNumDequant);
+      mbar_init(&B.afull[i], kNumDequant / 2);  // the warps of the group filling it
       mbar_init(&B.aempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -236,59 +236,60 @@ __global__ void __launch_bounds__(kThreadsTC, 1) tc_expert_kernel(const __grid_c
     }
     __syncwarp();
   } else if (warp < kWarpEpi0) {
-    // ---- dequant warps: 4 per TMEM lane quadrant (the quadrant holds units 2q, 2q + 1 of each M tile):
-    // with two M tiles one whole unit each, with one tile half a unit (2 of its 4 blocks) each ----
+    // ---- dequant warps: two groups of 8 take alternate K chunks, so that one group's barrier waits and
+    // tensor-memory stores overlap the other group's decode.  In a group, 2 warps per TMEM lane quadrant (the
+    // quadrant holds units 2q, 2q + 1 of each M tile), each decoding its unit in every M tile of the chunk ----
     const int dw = warp - kWarpDequant0;
-    const int q = warp & 3, uq = (dw >> 2) & 1;
-    const int m = kMT == 2 ? dw >> 3 : 0;
-    const int bb0 = kMT == 2 ? 0 : 2 * (dw >> 3);
-    constexpr int kNB = C::kBlocksPerWarp;
+    const int grp = dw >> 3, q = warp & 3, uq = (dw >> 2) & 1;
     const int unit = 2 * q + uq;
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * uq) << 16;
     const int g = lane >> 2;
     int cnt = 0;
     for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
       for (int kc = 0; kc < a.kchunks; ++kc, ++cnt) {
+        if ((cnt & 1) != grp) continue;
         const int s = cnt % kStages, sa = cnt % kAStages;
         waitb(&B.full[s], (cnt / kStages) & 1, B, a.status);
-        const uint8_t *gp = smem + s * kStageBytes + (m * kTileUnits + unit) * kGroupBytes;
-        const uint4 cw = *reinterpret_cast<const uint4 *>(gp + lane * 16);
-        const uint4 sw = *reinterpret_cast<const uint4 *>(gp + kGroupCodeBytes + g * 16);
-        const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
-        const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
-        // the whole unit in registers before the A stage is free: registers P0, P2 belong to row g,
-        // P1, P3 to row g+8
-        uint32_t av[kNB][8];
+        const uint32_t acol = tbase + lane_base + kTmemA0 + sa * kMT * 64;
+#pragma unroll 1
+        for (int m = 0; m < kMT; ++m) {
+          const uint8_t *gp = smem + s * kStageBytes + (m * kTileUnits + unit) * kGroupBytes;
+          const uint4 cw = *reinterpret_cast<const uint4 *>(gp + lane * 16);
+          const uint4 sw = *reinterpret_cast<const uint4 *>(gp + kGroupCodeBytes + g * 16);
+          const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+          const uint32_t sws[4] = {sw.x, sw.y, sw.z, sw.w};
+          // registers P0, P2 belong to row g, P1, P3 to row g+8
+          uint32_t av[4][8];
 #pragma unroll
-        for (int bb = 0; bb < kNB; ++bb) {
-          uint32_t p[8];
-          const uint32_t cword = kNB == 4 ? cws[bb] : (bb0 == 0 ? cws[bb] : cws[2 + bb]);
-          const uint32_t sword = kNB == 4 ? sws[bb] : (bb0 == 0 ? sws[bb] : sws[2 + bb]);
-          decode_q2_exact(cword, p);
-          uint32_t sg, sg8;
-          scale_pairs(sword, sg, sg8);
-          av[bb][0] = bf16x2_mul(p[0], sg);
-          av[bb][1] = bf16x2_mul(p[2], sg);
-          av[bb][2] = bf16x2_mul(p[1], sg8);
-          av[bb][3] = bf16x2_mul(p[3], sg8);
-          av[bb][4] = bf16x2_mul(p[4], sg);
-          av[bb][5] = bf16x2_mul(p[6], sg);
-          av[bb][6] = bf16x2_mul(p[5], sg8);
-          av[bb][7] = bf16x2_mul(p[7], sg8);
-        }
-        waitb(&B.aempty[sa], ((cnt / kAStages) & 1) ^ 1, B, a.status);
-        // The MMAs of chunk cnt - kAStages have completed (the commit that freed this A stage
-        // follows them): their shared-memory stage, whose codes this warp read long ago, is free.
-        if (cnt >= kAStages) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B.empty[(cnt - kAStages) % kStages]);
-        }
-        tc_fence_after();
-        const uint32_t acol = tbase + lane_base + kTmemA0 + (sa * kMT + m) * 64;
+          for (int bb = 0; bb < 4; ++bb) {
+            uint32_t p[8];
+            decode_q2_exact(cws[bb], p);
+            uint32_t sg, sg8;
+            scale_pairs(sws[bb], sg, sg8);
+            av[bb][0] = bf16x2_mul(p[0], sg);
+            av[bb][1] = bf16x2_mul(p[2], sg);
+            av[bb][2] = bf16x2_mul(p[1], sg8);
+            av[bb][3] = bf16x2_mul(p[3], sg8);
+            av[bb][4] = bf16x2_mul(p[4], sg);
+            av[bb][5] = bf16x2_mul(p[6], sg);
+            av[bb][6] = bf16x2_mul(p[5], sg8);
+            av[bb][7] = bf16x2_mul(p[7], sg8);
+          }
+          if (m == 0) {
+            waitb(&B.aempty[sa], ((cnt / kAStages) & 1) ^ 1, B, a.status);
+            // The MMAs of chunk cnt - kAStages (this group's previous chunk) have completed (the commit that
+            // freed this A stage follows them): their shared-memory stage, whose codes this group read, is free.
+            if (cnt >= kAStages) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&B.empty[(cnt - kAStages) % kStages]);
+            }
+            tc_fence_after();
+          }
 #pragma unroll
-        for (int bb = 0; bb < kNB; ++bb) {
-          tmem_st_16x256b(acol + 16 * (bb0 + bb), av[bb][0], av[bb][1], av[bb][2], av[bb][3]);
-          tmem_st_16x256b(acol + 16 * (bb0 + bb) + 8, av[bb][4], av[bb][5], av[bb][6], av[bb][7]);
+          for (int bb = 0; bb < 4; ++bb) {
+            tmem_st_16x256b(acol + m * 64 + 16 * bb, av[bb][0], av[bb][1], av[bb][2], av[bb][3]);
+            tmem_st_16x256b(acol + m * 64 + 16 * bb + 8, av[bb][4], av[bb][5], av[bb][6], av[bb][7]);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
