@@ -44,6 +44,7 @@ EXPORTED = [
     "moe_route",
     "moe_route_noalloc",
     "moe_layer_forward",
+    "moe_layer_forward_host",
     "moe_layer_forward_residual",
     "moe_experts_forward",
     "moe_dispatch",
@@ -79,6 +80,9 @@ def lib():
         L.moe_layer_forward.restype = ctypes.c_int
         L.moe_layer_forward.argtypes = [D, P, ctypes.POINTER(moe_router), ctypes.POINTER(moe_experts),
                                         ctypes.POINTER(moe_shared), P, i32, P, P, P, sz, P]
+        L.moe_layer_forward_host.restype = ctypes.c_int
+        L.moe_layer_forward_host.argtypes = [D, P, ctypes.POINTER(moe_router), ctypes.POINTER(moe_experts),
+                                             ctypes.POINTER(moe_shared), P, i32, P, P, P, sz, P]
         L.moe_layer_forward_residual.restype = ctypes.c_int
         L.moe_layer_forward_residual.argtypes = [D, P, ctypes.POINTER(moe_router), ctypes.POINTER(moe_experts),
                                                  ctypes.POINTER(moe_shared), P, P, ctypes.c_float, i32, P, P, P, sz,
@@ -177,6 +181,19 @@ def moe_layer_forward(dims, x, router_w, router_b, experts_packed, shared_packed
                                    ctypes.byref(sh), _ptr(out), int(T), _ptr(topk_idx_out), _ptr(topk_w_out),
                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "moe_layer_forward")
+
+
+def moe_layer_forward_host(dims, x_host, router_w, router_b, experts_packed, shared_packed, out_host, T: int,
+                           workspace, topk_idx_out=None, topk_w_out=None, stream=None):
+    """x_host / out_host: page-locked host tensors (e.g. torch's pin_memory()), T <= 8."""
+    r = moe_router(_ptr(router_w), _ptr(router_b))
+    ex = moe_experts(_ptr(experts_packed))
+    sh = moe_shared(_ptr(shared_packed))
+    code = lib().moe_layer_forward_host(ctypes.byref(_dims(dims)), _ptr(x_host), ctypes.byref(r), ctypes.byref(ex),
+                                        ctypes.byref(sh), _ptr(out_host), int(T), _ptr(topk_idx_out),
+                                        _ptr(topk_w_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream))
+    _check(code, "moe_layer_forward_host")
 
 
 def moe_layer_forward_residual(dims, x_norm_in, router_w, router_b, experts_packed, shared_packed, resid, x_norm_out,

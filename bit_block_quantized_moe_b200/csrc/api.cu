@@ -66,6 +66,8 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
   const size_t o_wsplit = take(rtc ? (size_t)3 * E * H * 2 : 0);
   // sized by the bound on every T (the split count falls as T grows), so that a workspace sized for max_T fits
   const size_t o_rpart = take(rtc ? router_tc_partial_bytes_max() : 0);
+  const size_t host_rows = (size_t)(T < kHostIoMaxTokens ? T : kHostIoMaxTokens) * H * 2;
+  const size_t o_hx = take(host_rows), o_hy = take(host_rows);
   if (base && ws) {
     uint8_t *b = static_cast<uint8_t *>(base);
     ws->status = reinterpret_cast<uint32_t *>(b + o_hdr);
@@ -96,6 +98,8 @@ size_t workspace_layout(const moe_dims &d, int T, void *base, Workspace *ws) {
     ws->partial = reinterpret_cast<float *>(b + o_part);
     ws->wsplit = rtc ? reinterpret_cast<uint16_t *>(b + o_wsplit) : nullptr;
     ws->rpart = reinterpret_cast<float *>(b + o_rpart);
+    ws->host_x = reinterpret_cast<uint16_t *>(b + o_hx);
+    ws->host_y = reinterpret_cast<uint16_t *>(b + o_hy);
     ws->words = (int)words;
     ws->max_items = max_items;
   }
@@ -267,6 +271,32 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
   LayerOut lo;
   lo.out = out;
   return cuda_status(run_layer(*dims, x, router, experts, shared, lo, T, topk_idx_out, topk_w_out, ws, s));
+}
+
+moe_status moe_layer_forward_host(const moe_dims *dims, const uint16_t *x_host, const moe_router *router,
+                                  const moe_experts *experts, const moe_shared *shared, uint16_t *out_host,
+                                  int32_t T, int32_t *topk_idx_out, float *topk_w_out, void *workspace,
+                                  size_t ws_bytes, moe_stream_t stream) {
+  if (!router) return MOE_ERR_ARG;
+  moe_status st = check_layer_args(dims, x_host, experts, shared, out_host, T, workspace, ws_bytes);
+  if (st != MOE_OK || T == 0) return st;
+  if (T > kHostIoMaxTokens || !router->w) return MOE_ERR_ARG;
+  if (!aligned16(router->w)) return MOE_ERR_ALIGN;
+  const moe_status dev = device_ok();
+  if (dev != MOE_OK) return dev;
+  const size_t rows = (size_t)T * dims->hidden * 2;
+  void *xd = mapped_host_range(x_host, rows), *od = mapped_host_range(out_host, rows);
+  if (!xd || !od) return MOE_ERR_ARG;  // not page-locked, device-mapped host memory: nothing launched
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Workspace ws;
+  workspace_layout(*dims, T, workspace, &ws);
+  LayerOut lo;
+  lo.out = ws.host_y;
+  cudaError_t err = launch_stream_copy16(xd, ws.host_x, rows, s);
+  if (err == cudaSuccess)
+    err = run_layer(*dims, ws.host_x, router, experts, shared, lo, T, topk_idx_out, topk_w_out, ws, s);
+  if (err == cudaSuccess) err = launch_stream_copy16(ws.host_y, od, rows, s);
+  return cuda_status(err);
 }
 
 static bool overlaps(const void *a, size_t na, const void *b, size_t nb) {

@@ -33,6 +33,8 @@ struct Workspace {
   float *partial;          // fused decode: per (expert, tile) partial outputs
   uint16_t *wsplit;        // tcgen05 router: [3][E][H] bf16 planes of the router weights (null: legacy router)
   float *rpart;            // tcgen05 router: [ksplit][T][E] K-split partial logits (ksplit > 1)
+  uint16_t *host_x;        // moe_layer_forward_host: [min(T, 8)][H] bf16 token rows staged from host memory
+  uint16_t *host_y;        // moe_layer_forward_host: [min(T, 8)][H] bf16 layer output staged for host memory
   int words;               // ceil(T / 32)
   int max_items;
   int max_tc_items;
@@ -78,5 +80,10 @@ cudaError_t launch_rmsnorm_residual_f32(float *resid, const float *y, uint16_t *
                                         cudaStream_t s);
 cudaError_t launch_combine_rmsnorm(const moe_dims &d, int T, const Workspace &ws, float *resid, uint16_t *x_norm,
                                    float eps, cudaStream_t s);
+// Host-memory token rows (hostio.cu): a one-kernel 16-byte copy in stream order (programmatic dependent launch,
+// nothing touched before the wait), and the device address of a page-locked, device-mapped host range.
+constexpr int kHostIoMaxTokens = 8;
+cudaError_t launch_stream_copy16(const void *src, void *dst, size_t bytes, cudaStream_t s);
+void *mapped_host_range(const void *p, size_t bytes);
 
 }  // namespace moe

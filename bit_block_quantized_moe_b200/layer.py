@@ -71,6 +71,17 @@ class Q2MoeLayer:
                             self.workspace, topk_idx, topk_w, stream)
         return out
 
+    def forward_host(self, x_host, out_host=None, topk_idx=None, topk_w=None, stream=None):
+        """x_host: [T <= 8, hidden] bf16 bit patterns in page-locked host memory; the output goes to out_host
+        (page-locked, allocated if None), complete once the stream has passed the call."""
+        T = x_host.shape[0]
+        self.reserve(T)
+        if out_host is None:
+            out_host = torch.empty(x_host.shape, dtype=x_host.dtype).pin_memory()
+        B.moe_layer_forward_host(self.dims, x_host, self.router_w, self.router_b, self.experts, self.shared, out_host,
+                                 T, self.workspace, topk_idx, topk_w, stream)
+        return out_host
+
     def forward_residual(self, x_norm, resid, x_norm_out, eps=1e-6, topk_idx=None, topk_w=None, stream=None):
         """One stacked layer: resid += layer(x_norm); x_norm_out = bf16(RMSNorm(resid))."""
         T = x_norm.shape[0]

@@ -198,6 +198,27 @@ moe_status moe_layer_forward(const moe_dims *dims, const uint16_t *x, const moe_
                              int32_t *topk_idx_out, float *topk_w_out, void *workspace, size_t ws_bytes,
                              moe_stream_t stream);
 
+/* ---- layer forward, token rows in host memory ----------------------------------
+ * Host.  The layer of moe_layer_forward for a decode window (1 <= T <= 8)
+ * whose token rows live in page-locked host memory, as in a serving loop that
+ * hands the layer one window at a time: x_host [T, hidden] bf16 is read and
+ * out_host [T, hidden] bf16 written by the library's own kernels over the
+ * host link (zero-copy), in stream order with the layer, so that no copy call
+ * of the caller's sits between them.  Both must be page-locked host memory
+ * mapped into the device's address space (cudaHostAlloc / cudaMallocHost, or
+ * cudaHostRegister with the mapped flag, on a unified-address system), each
+ * range within one allocation, 16-byte aligned and not overlapping; anything
+ * else returns MOE_ERR_ARG (MOE_ERR_ALIGN for alignment) before any launch,
+ * as does T > 8.  The rows are staged in the workspace (moe_workspace_bytes
+ * covers them).  out_host holds the result once the stream has passed this
+ * call (e.g. after cudaStreamSynchronize).  Other arguments, the routing
+ * copies and the errors are those of moe_layer_forward, whose output this
+ * equals bit for bit. */
+moe_status moe_layer_forward_host(const moe_dims *dims, const uint16_t *x_host, const moe_router *router,
+                                  const moe_experts *experts, const moe_shared *shared, uint16_t *out_host,
+                                  int32_t T, int32_t *topk_idx_out, float *topk_w_out, void *workspace,
+                                  size_t ws_bytes, moe_stream_t stream);
+
 /* One layer of a stack of layers (the pages' model stacks 48 of them, Strata
  * tuning page, section 2 model table), with the residual stream and the next
  * layer's normalisation done by the layer's own last kernel:

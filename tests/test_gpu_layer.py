@@ -263,6 +263,50 @@ def test_fused_decode_barrier_counter(full):
         check_layer(CONFIGS["prefill"], w, x, y, idx, wts)
 
 
+def test_layer_forward_host_memory(full):
+    """moe_layer_forward_host: the token rows read from and the output written to page-locked host memory by
+    the library's copy kernels in stream order, equal bit for bit to moe_layer_forward on device buffers
+    (routing copies too); several steps back to back on one stream with no synchronisation between them (the
+    copy-in of a step is launched while the previous step still runs) and each against the oracle."""
+    from bit_block_quantized_moe_b200 import MoeError, moe_layer_forward_host
+
+    L, w = full
+    L.reserve(8)
+    stream = torch.cuda.Stream()
+    steps = [(3, 301), (1, 302), (8, 303), (3, 304), (2, 305)]
+    xh = [torch.from_numpy(make_x(T, 2048, seed=sd).view(np.int16)).pin_memory() for T, sd in steps]
+    oh = [torch.zeros((T, 2048), dtype=torch.int16).pin_memory() for T, _ in steps]
+    ih = [torch.full((T, 10), -1, dtype=torch.int32, device="cuda") for T, _ in steps]
+    wh = [torch.zeros((T, 10), dtype=torch.float32, device="cuda") for T, _ in steps]
+    with torch.cuda.stream(stream):
+        for i in range(len(steps)):
+            L.forward_host(xh[i], oh[i], topk_idx=ih[i], topk_w=wh[i], stream=stream)
+    stream.synchronize()
+    L.check_status()
+    for i, (T, _) in enumerate(steps):
+        x = xh[i].numpy()
+        y_ref, idx_ref, w_ref = gpu_forward(L, x)
+        y = bf16_to_f32(oh[i].numpy()).astype(np.float64)
+        assert np.array_equal(y, y_ref), T
+        assert np.array_equal(ih[i].cpu().numpy(), idx_ref) and np.array_equal(wh[i].cpu().numpy(), w_ref)
+        check_layer(CONFIGS["prefill"], w, x.view(np.uint16), y, idx_ref, w_ref)
+    # pageable host memory, device memory and windows over 8 tokens are refused before any launch
+    pageable = torch.from_numpy(make_x(3, 2048, seed=1).view(np.int16))
+    for bad_x, bad_out, T in ((pageable, oh[0], 3), (xh[0], torch.zeros((3, 2048), dtype=torch.int16), 3),
+                              (xh[0].cuda(), oh[0], 3)):
+        with pytest.raises(MoeError) as e:
+            moe_layer_forward_host(L.dims, bad_x, L.router_w, L.router_b, L.experts, L.shared, bad_out, T,
+                                   L.workspace)
+        assert e.value.code == 1  # MOE_ERR_ARG
+    x9 = torch.from_numpy(make_x(9, 2048, seed=2).view(np.int16)).pin_memory()
+    o9 = torch.zeros((9, 2048), dtype=torch.int16).pin_memory()
+    L.reserve(9)
+    with pytest.raises(MoeError) as e:
+        moe_layer_forward_host(L.dims, x9, L.router_w, L.router_b, L.experts, L.shared, o9, 9, L.workspace)
+    assert e.value.code == 1
+    L.check_status()
+
+
 @pytest.mark.parametrize("T", [4, 5, 8])
 def test_fused_decode_window_sizes(full, T):
     L, w = full
