@@ -88,6 +88,28 @@ def test_host_checks_before_launch(lib):
     assert lib.moe_rmsnorm_residual(None, None, None, 4, 256, 1e-6, None) == 1
 
 
+def test_host_memory_entry_point_checks(lib):
+    """moe_layer_forward_host: the same argument checks as moe_layer_forward, and windows over 8 tokens refused,
+    all before the device is touched (the host pointers here are never dereferenced)."""
+    d = B.moe_dims(256, 128, 16, 2)
+    r = B.moe_router(0x1000, None)
+    ex, sh = B.moe_experts(0x2000), B.moe_shared(0x3000)
+
+    def call(x=0x4000, out=0x8000, T=8, wsp=0x10000, wsb=None):
+        wsb = B.moe_workspace_bytes(d, max(T, 1)) if wsb is None else wsb
+        return lib.moe_layer_forward_host(ctypes.byref(d), x, ctypes.byref(r), ctypes.byref(ex), ctypes.byref(sh),
+                                          out, T, None, None, wsp, wsb, None)
+
+    assert call(T=0) == 0
+    assert call(T=-1) == 1
+    assert call(T=9) == 1                      # only decode windows
+    assert call(x=0x4008) == 2
+    assert call(wsb=16) == 3
+    assert call(out=0x4000 + 256) == 1
+    # the staging rows are part of the workspace: one sized for T holds every T' <= T
+    assert B.moe_workspace_bytes(d, 8) >= B.moe_workspace_bytes(d, 3) > 0
+
+
 @pytest.mark.parametrize("dims", [(2048, 512, 512, 10), (256, 128, 16, 2), (512, 512, 16, 2), (4096, 4096, 4096, 32),
                                   (256, 1024, 4096, 8)])
 def test_workspace_size_never_shrinks_with_tokens(lib, dims):
