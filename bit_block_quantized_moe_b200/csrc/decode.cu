@@ -26,8 +26,10 @@
 //     own shared-memory slot in four cp.async groups, keeps the next two
 //     quarters in flight while it computes, runs the whole unit (full K) with
 //     no cross-warp reduction and writes h = silu(g) * u (bf16) straight from
-//     its accumulators.  At the end the CTA publishes, per expert, how many of
-//     its units are done.
+//     its accumulators.  For one token (fewer units than warps) the kernel
+//     instance <2, 1> splits each unit's K over two warps, whose sums meet in
+//     shared memory in part order, and gives each down stage one unit.  At the
+//     end the CTA publishes, per expert, how many of its units are done.
 //  D  Once the h of the (at most two) experts in the CTA's down range is
 //     complete (per-expert counter, bounded wait) it is copied into shared
 //     memory; each down stage (two 16-row units) again belongs to one warp:
@@ -63,6 +65,7 @@ constexpr int kSlotTokens = 3;            // up to this many tokens: one work en
 constexpr int kMaxE = 1024;
 constexpr int kMaxI = 512;                // down K handled by the h cache
 constexpr int kBarConsumers = 1;          // named barrier id (0 = __syncthreads)
+constexpr int kMaxParts = 40;             // gate/up K parts a CTA may hold in shared memory (128 floats each)
 
 struct DecodeArgs {
   const uint16_t *x;
@@ -93,7 +96,7 @@ struct SmemLayout {
 
 __host__ __device__ inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes) {
+__host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t stage_bytes, int kp) {
   SmemLayout L;
   uint32_t o = 0;
   L.xs = o;  // [T + 1][H + 16] bf16 token rows (the B operand once prepared); row T stays zero
@@ -105,8 +108,11 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int H, int ns, uint32_t
   L.rpart = o;  // [rows per pass][8 tokens][router parts]
   o += (kConsumerWarps / kRouterParts) * kMaxTok * kRouterParts * 4;
   o = align_to(o, 16);
-  L.red = o;  // top-k scratch (phase B: 64 uint64 per token), then the h staging of phase D: [2][T][I + 16] bf16
-  o += align_to(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), 16);
+  // top-k scratch (phase B: 64 uint64 per token), the gate/up K parts at the end of phase C (kp > 1:
+  // [unit][part][32 lanes][4] floats), then the h staging of phase D: [2][T][I + 16] bf16
+  L.red = o;
+  const uint32_t parts_bytes = kp > 1 ? (uint32_t)kMaxParts * 128 * 4 : 0u;
+  o += align_to(max(max((uint32_t)kMaxTok * 64 * 8, 2u * T * (kMaxI + 16) * 2), parts_bytes), 16);
   L.bitmap = o;
   o += (kMaxE / 32) * 4;
   L.slv = o;  // slot entries: the winners' logits, token-major
@@ -199,11 +205,13 @@ __device__ __forceinline__ void unit_gemv(const uint8_t *st, int grp0, int grp1,
   }
 }
 
+template <int KP, int PPS>
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a) {
+  static_assert((KP == 1 || KP == 2 || KP == 4) && (PPS == 1 || PPS == 2), "work granularity");
   extern __shared__ __align__(128) uint8_t smem[];
   const PackedGeom &G = a.G;
   const int T = a.T, E = a.E, K = a.k, H = G.H, I = G.I;
-  const SmemLayout L = smem_layout(T, H, a.ns, a.stage_bytes);
+  const SmemLayout L = smem_layout(T, H, a.ns, a.stage_bytes, KP);
   uint16_t *xs = reinterpret_cast<uint16_t *>(smem + L.xs);
   float *corr = reinterpret_cast<float *>(smem + L.corr);
   float *hcorr = reinterpret_cast<float *>(smem + L.hcorr);
@@ -386,49 +394,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   __syncthreads();  // the list is visible to every warp
 
   const int nent = misc[0];
+  const int nw = a.nw;
   const int n_gu = nent * G.gu_units, n_dn = nent * G.dn_units;
   // contiguous shares of the units (32-bit products: at most 129 entries x 256 units x the grid)
   const int g0 = (int)((uint32_t)n_gu * blockIdx.x / gridDim.x);
   const int g1 = (int)((uint32_t)n_gu * (blockIdx.x + 1) / gridDim.x);
   const int d0 = (int)((uint32_t)n_dn * blockIdx.x / gridDim.x);
   const int d1 = (int)((uint32_t)n_dn * (blockIdx.x + 1) / gridDim.x);
-  const int pps = 2;  // down units (16 rows) per stage: enough stages to keep every warp busy
-  const int n_gu_st = g1 - g0;
+  // Granularity (compile-time, chosen by the launcher): a gate/up unit's K is split into kp parts on
+  // different warps (stages of a quarter of the part each), summed in part order before SwiGLU, and a down
+  // stage holds pps units (quarters of half or a quarter of a unit).
+  constexpr int kp = KP, pps = PPS;
+  constexpr int qpu = 4 / pps;  // quarters per down unit
+  const int n_gu_st = (g1 - g0) * kp;
   const int n_dn_st = (d1 - d0 + pps - 1) / pps;
   const int n_st = n_gu_st + n_dn_st;
   // Stage s belongs to warp s % nw, which copies it (cp.async) into its own
   // ring slot, waits for its own copies, computes it and refills the slot with
   // its next stage s + nw.  No other warp touches the slot.
-  const int nw = a.nw;
   auto expert_ptr = [&](int entry) -> const uint8_t * {
     const int e = ent[entry];
     return e == E ? a.shared : a.experts + (size_t)e * G.expert_bytes;
   };
   auto stage_ptr = [&](int) { return ring + (size_t)warp * a.stage_bytes; };
-  // A stage is copied as 4 commit groups (its quarters): gate/up = one unit
-  // (quarter = 4 block groups), down = 2 units of 16 rows (quarter = half a
-  // unit).  A warp walks the quarters of its stages in order and keeps the next
-  // two in flight: quarter i is computed after quarter i + 1 was issued, and
-  // quarter i + 2 goes into the slot region quarter i - 2 used.  Past the last
-  // stage the groups are empty.
+  // A stage is copied as 4 commit groups (its quarters): gate/up = one unit, or
+  // one of its kp K parts (quarter = 4 / kp block groups), down = pps units of
+  // 16 rows (quarter = half a unit, or a quarter with one unit).  A warp walks
+  // the quarters of its stages in order and keeps the next two in flight:
+  // quarter i is computed after quarter i + 1 was issued, and quarter i + 2 goes
+  // into a slot region that overlaps none of quarter i + 1's (the region
+  // quarter i used, or for the first down quarters the first gate/up ones').
+  // Past the last stage the groups are empty.
   auto issue_quarter = [&](int qi) {
     const int s = warp + (qi >> 2) * nw, qt = qi & 3;
     if (s < n_st) {
       uint8_t *dst = stage_ptr(s);
       if (s < n_gu_st) {
-        const int id = g0 + s;
-        const size_t qb = G.gu_unit_bytes / 4;
+        const int id = g0 + s / kp, part = s % kp;
+        const size_t qb = G.gu_unit_bytes / (4 * kp);
         warp_cp_async(dst + qt * qb,
-                      expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes + qt * qb,
+                      expert_ptr(id / G.gu_units) + (size_t)(id % G.gu_units) * G.gu_unit_bytes +
+                          (size_t)(4 * part + qt) * qb,
                       (uint32_t)qb, lane);
       } else {
-        const int q = d0 + (s - n_gu_st) * pps + (qt >> 1);
-        const size_t hb2 = G.dn_unit_bytes / 2;
+        const int q = d0 + (s - n_gu_st) * pps + qt / qpu, piece = qt % qpu;
+        const size_t pb = G.dn_unit_bytes / qpu;
         if (q < d1)
-          warp_cp_async(dst + (size_t)(qt >> 1) * G.dn_unit_bytes + (qt & 1) * hb2,
+          warp_cp_async(dst + (size_t)(qt / qpu) * G.dn_unit_bytes + piece * pb,
                         expert_ptr(q / G.dn_units) + G.gu_bytes + (size_t)(q % G.dn_units) * G.dn_unit_bytes +
-                            (qt & 1) * hb2,
-                        (uint32_t)hb2, lane);
+                            piece * pb,
+                        (uint32_t)pb, lane);
       }
     }
     cp_async_commit();
@@ -450,16 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
   }
 
   // ---------------- consumers, phase C: gate/up + SwiGLU ----------------
-  for (int s_idx = warp; warp < nw && s_idx < n_gu_st; s_idx += nw) {
-    const uint8_t *st = stage_ptr(s_idx);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int gq = G.gu_groups / 4;  // block groups per quarter
-    for (int qt = 0; qt < 4; ++qt) {
-      next_quarter();
-      unit_gemv(st, qt * gq, (qt + 1) * gq, xs, xstride, T, zrow, corr, lane, acc);
-      done_quarter();
-    }
-    const int id = g0 + s_idx;
+  // h = silu(gate) * up of unit id from its accumulators (rows g and g+8, tokens 2c and 2c + 1).
+  auto write_h = [&](int id, const float (&acc)[4]) {
     const int entry = id / G.gu_units, u = id % G.gu_units;
     const int i = 8 * u + g;  // tile rows g (gate) and g+8 (up) share intermediate row i
 #pragma unroll
@@ -469,6 +476,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
         const int j = tokj[entry * kMaxTok + n];
         if (j >= 0) a.h[((size_t)n * (K + 1) + j) * I + i] = float_to_bf16_bits(silu_f(acc[hf]) * acc[2 + hf]);
       }
+    }
+  };
+  for (int s_idx = warp; warp < nw && s_idx < n_gu_st; s_idx += nw) {
+    const uint8_t *st = stage_ptr(s_idx);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int gq = G.gu_groups / (4 * kp);     // block groups per quarter
+    const int k0 = (s_idx % kp) * 4 * gq;      // the part's first block group along K
+    for (int qt = 0; qt < 4; ++qt) {
+      next_quarter();
+      unit_gemv(st - (size_t)k0 * kGroupBytes, k0 + qt * gq, k0 + (qt + 1) * gq, xs, xstride, T, zrow, corr, lane,
+                acc);
+      done_quarter();
+    }
+    if constexpr (kp == 1)
+      write_h(g0 + s_idx, acc);
+    else  // the part's sums into [unit][part][32 lanes][4] (the top-k scratch is free, the h cache not yet used)
+      *reinterpret_cast<float4 *>(red + (size_t)s_idx * 128 + lane * 4) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+  if constexpr (kp > 1) {
+    named_bar(kBarConsumers, kConsumers);
+    for (int ul = warp; ul < g1 - g0; ul += kConsumerWarps) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int p = 0; p < kp; ++p) {
+        const float4 v = *reinterpret_cast<const float4 *>(red + (size_t)(ul * kp + p) * 128 + lane * 4);
+        acc[0] += v.x;
+        acc[1] += v.y;
+        acc[2] += v.z;
+        acc[3] += v.w;
+      }
+      write_h(g0 + ul, acc);
     }
   }
 
@@ -576,10 +614,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
       const uint16_t *hrows = hc + he * T * hstride;
       const float *hce = hcorr + he * (kMaxI / 32) * kMaxTok;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int hg = G.dn_groups / 2;  // block groups per half unit
-      for (int h2 = 0; h2 < 2; ++h2) {
+      const int hg = G.dn_groups / qpu;  // block groups per quarter
+      for (int hq = 0; hq < qpu; ++hq) {
         next_quarter();
-        if (live) unit_gemv(pp_st, h2 * hg, (h2 + 1) * hg, hrows, hstride, T, zrow, hce, lane, acc);
+        if (live) unit_gemv(pp_st, hq * hg, (hq + 1) * hg, hrows, hstride, T, zrow, hce, lane, acc);
         done_quarter();
       }
       if (!live) continue;
@@ -610,8 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(DecodeArgs a)
 constexpr int kMaxDevices = 64;
 struct LaunchCache {
   std::atomic<int> n_sm{0}, max_smem{0};
-  std::atomic<uint32_t> checked_smem{0};  // shared-memory size whose residency was checked (0: none)
-  uint32_t smem_attr = 0;                 // largest dynamic shared memory opted into (under mu)
+  // per kernel instance (0: <1, 2>, 1: <2, 1>)
+  std::atomic<uint32_t> checked_smem[2] = {{0u}, {0u}};  // shared-memory size whose residency was checked (0: none)
+  uint32_t smem_attr[2] = {0u, 0u};                        // largest dynamic shared memory opted into (under mu)
   std::mutex mu;
 };
 LaunchCache g_launch_cache[kMaxDevices];
@@ -652,12 +691,18 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
     lc.n_sm.store(n_sm, std::memory_order_release);
   }
   const uint32_t stage_bytes = (uint32_t)max(G.gu_unit_bytes, 4 * G.dn_unit_bytes);
-  const SmemLayout L0 = smem_layout(T, G.H, 0, stage_bytes);
+  // Work granularity.  One token gives a CTA fewer gate/up units than warps (4.75 of 14 at the pages' shape): that
+  // instance splits each unit's K over two warps and gives each down stage one unit (21.2 -> 19.6 us per step on
+  // B200); every other window keeps whole units and two-unit down stages.
+  const int gu_cta = ((min(T * d.top_k, d.n_experts) + 1) * G.gu_units + n_sm - 1) / n_sm;
+  const int inst = (T == 1 && G.gu_groups % 8 == 0 && gu_cta * 2 <= kMaxParts) ? 1 : 0;
+  const int kp = inst ? 2 : 1;
+  const SmemLayout L0 = smem_layout(T, G.H, 0, stage_bytes, kp);
   const int slots = (int)((max_smem - (int)L0.ring - 128) / (int)stage_bytes);
   if (slots < 1) return cudaErrorInvalidConfiguration;
   const int nw = min(kConsumerWarps, slots);  // warps streaming and computing stages, one slot each
   const int ns = nw;
-  const SmemLayout L = smem_layout(T, G.H, ns, stage_bytes);
+  const SmemLayout L = smem_layout(T, G.H, ns, stage_bytes, kp);
   if (L.total > (uint32_t)max_smem) return cudaErrorInvalidConfiguration;
   // a CTA's down range spans at most two entries (the h cache of phase D holds two): at most dn_units units
   const int max_entries = min(T * d.top_k, d.n_experts) + 1;
@@ -690,21 +735,21 @@ cudaError_t launch_decode_fused(const moe_dims &d, const uint16_t *x, const floa
   a.nw = nw;
   a.stage_bytes = stage_bytes;
 
-  void (*kern)(DecodeArgs) = decode_fused_kernel;
-  // The shared-memory opt-in and the residency check are done once per device and shared-memory size
-  // (they depend on nothing else), not on every call.
-  if (lc.checked_smem.load(std::memory_order_acquire) != L.total) {
+  void (*kern)(DecodeArgs) = inst ? decode_fused_kernel<2, 1> : decode_fused_kernel<1, 2>;
+  // The shared-memory opt-in and the residency check are done once per device, instance and shared-memory
+  // size (they depend on nothing else), not on every call.
+  if (lc.checked_smem[inst].load(std::memory_order_acquire) != L.total) {
     std::lock_guard<std::mutex> lock(lc.mu);
-    if (L.total > lc.smem_attr) {
+    if (L.total > lc.smem_attr[inst]) {
       err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
       if (err != cudaSuccess) return err;
-      lc.smem_attr = L.total;
+      lc.smem_attr[inst] = L.total;
     }
     int per_sm = 0;
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, L.total);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    lc.checked_smem.store(L.total, std::memory_order_release);
+    lc.checked_smem[inst].store(L.total, std::memory_order_release);
   }
 
   cudaLaunchConfig_t cfg{};
